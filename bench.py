@@ -1,0 +1,500 @@
+#!/usr/bin/env python3
+"""Benchmark of the MoE layout -> dispatch -> combine hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline] [--no-e2e]
+
+A step is one pass of the whole path over one batch: ep_layout (3 kernels),
+ep_dispatch (FP8 e4m3 or BF16), ep_combine (BF16), all through the C ABI.
+The default workload is the one the metric is quoted on: 8192 tokens,
+hidden 7168, top-8 of 256 experts with group-limited gating (8 groups, top-4
+groups, Zipf(1.0) bias), 64 virtual ranks, FP8 dispatch, BF16 combine.
+
+Timing: inputs resident in HBM; L2 flushed (256 MiB write) before every
+timed step; CUDA events on the launching stream around each call; W warm-up
+steps; K timed steps bracketed by barrier + synchronize; max over ranks.
+value = algorithmic bytes of all ranks' steps / time (GB/s).  Multi-GPU runs
+are independent replicas (each rank its own batch, seed + rank): the path
+has no exchange step on one node's virtual ranks, so there is no collective.
+
+`--impl reference` times the CPU oracle (the plain single-threaded C
+implementation under oracle/) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from combine_ep_layout_10_b200 import workloads as W  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+HBM_FALLBACK_GBS = 6650.0
+
+# DRAM traffic per launch from one ncu capture, keyed by the sha256 of the
+# kernel source it was taken on (stale -> reported as null).
+NCU_TRAFFIC = {}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=W.METRIC_WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (exact reads + writes each kernel must do)
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(w: W.Workload, V: int, n_rows: int) -> dict:
+    T, H, k, E, R = w.T, w.H, w.k, w.E, w.R
+    layout = T * k * 4 + E * 4 + R * 4 + T * R + T * k * 4 + n_rows * 4 + (E + 1) * 4 + (R + 1) * 4
+    if w.fp8:
+        dispatch = T * H * 2 + T * k * 4 + V * H + V * (H // 128) * 4
+    else:
+        dispatch = T * H * 2 + T * k * 4 + V * H * 2
+    combine = V * H * 2 + T * k * 4 + T * k * 4 + T * H * 2
+    return {"layout": layout, "dispatch": dispatch, "combine": combine,
+            "step": layout + dispatch + combine}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": HBM_FALLBACK_GBS, "source": "fallback"}
+
+
+def source_sha(name: str) -> str:
+    p = os.path.join(ROOT, "combine_ep_layout_10_b200", "csrc", name)
+    with open(p, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (n_gpus, world))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(orc, w: W.Workload, x, idx, tw, n_tok: int, y_sample):
+    """One oracle pass: full layout + dispatch/combine of the first n_tok tokens."""
+    _, L = orc.layout(idx, w.E, w.R, w.align, w.capacity)
+    pos = np.arange(n_tok * w.k, dtype=np.int32).reshape(n_tok, w.k)
+    if w.fp8:
+        orc.dispatch_fp8(x[:n_tok], pos, n_tok * w.k)
+    else:
+        orc.dispatch_bf16(x[:n_tok], pos, n_tok * w.k)
+    orc.combine(y_sample, tw[:n_tok], pos)
+    return L
+
+
+def oracle_sample_inputs(w, seed, n_tok):
+    x, idx, tw = W.make_routing(w, seed)
+    y = W.make_expert_out(n_tok * w.k, w.H, seed + 1)
+    return x, idx.numpy(), tw.numpy(), y
+
+
+def oracle_bytes(w, n_tok, n_rows_full):
+    sub = w.scaled(T=n_tok)
+    b = algorithmic_bytes(sub, n_tok * w.k, n_tok * w.k)
+    full_layout = algorithmic_bytes(w, w.T * w.k, n_rows_full)["layout"]
+    return full_layout + b["dispatch"] + b["combine"]
+
+
+def cpu_baseline(w: W.Workload, seed: int, budget_s: float = 12.0, n_tok: int = 2048) -> dict:
+    import oracle as orc
+    n_tok = min(n_tok, w.T)
+    x, idx, tw, y = oracle_sample_inputs(w, seed, n_tok)
+    n_rows = orc.max_recv_rows(w.T, w.k, w.E, w.align, w.capacity)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle_sample_step(orc, w, x, idx, tw, n_tok, y)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    byts = oracle_bytes(w, n_tok, n_rows) * reps
+    return {"value": byts / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d x (layout of all %d tokens + %s dispatch and BF16 combine of the first "
+                      "%d tokens), %.1f s single-threaded C" % (reps, w.T, "FP8" if w.fp8 else "BF16",
+                                                                 n_tok, dt),
+            "host_cpu": host_cpu()}
+
+
+def host_cpu() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return "%s x%d" % (ln.split(":", 1)[1].strip(), os.cpu_count() or 0)
+    except Exception:
+        pass
+    return "unknown"
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle as orc
+    n_tok = min(1024, w.T)
+    x, idx, tw, y = oracle_sample_inputs(w, args.seed, n_tok)
+    n_rows = orc.max_recv_rows(w.T, w.k, w.E, w.align, w.capacity)
+    for _ in range(args.warmup):
+        oracle_sample_step(orc, w, x, idx, tw, n_tok, y)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(orc, w, x, idx, tw, n_tok, y)
+    dt = time.perf_counter() - t0
+    byts = oracle_bytes(w, n_tok, n_rows) * args.steps
+    value = byts / dt / 1e9
+    sample = ("each step: layout of all %d tokens + %s dispatch and BF16 combine of the first %d "
+              "tokens (single-threaded C oracle)" % (w.T, "FP8" if w.fp8 else "BF16", n_tok))
+    line = {
+        "impl": "reference", "metric": "dispatch/combine HBM GB/s & % of peak; us/call at 8192 tok, "
+                                       "H=7168, top-8", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample, "host_cpu": host_cpu()},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: W.Workload, world: int) -> dict:
+    return {"workload": w.name, "tokens": w.T, "hidden": w.H, "topk": w.k, "experts": w.E,
+            "virtual_ranks": w.R, "dispatch": "fp8_e4m3 (fp32 scale / 128 ch)" if w.fp8 else "bf16",
+            "combine": "bf16 (fp32 fma chain)", "capacity": w.capacity, "expert_alignment": w.align,
+            "routing": w.routing, "l2": "flushed before every timed step (256 MiB write)",
+            "replicas": world, "parallelism": "replicas (no collective)"}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w):
+    from combine_ep_layout_10_b200 import build as B
+    from combine_ep_layout_10_b200 import ep
+
+    world, rank, local = dist_setup(args.gpus)
+    if not os.path.exists(ep.LIB_PATH):
+        B.build()
+    ep.lib()
+    dev = torch.device("cuda", local)
+    seed = args.seed + rank
+    x_cpu, idx_cpu, tw_cpu = W.make_routing(w, seed)
+    T, H, k, E, R = w.T, w.H, w.k, w.E, w.R
+    n_rows = ep.ep_max_recv_rows(T, k, E, w.align, w.capacity)
+    V = int((idx_cpu >= 0).sum())
+    nbytes = algorithmic_bytes(w, V, n_rows)
+
+    x = x_cpu.to(dev)
+    idx = idx_cpu.to(dev)
+    tw = tw_cpu.to(dev)
+    g = torch.Generator(device=dev).manual_seed(seed + 1)
+    y = torch.randn(n_rows, H, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    rdt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
+    recv = torch.empty(n_rows, H, dtype=rdt, device=dev)
+    scales = torch.empty(n_rows, H // 128, dtype=torch.float32, device=dev) if w.fp8 else None
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    cnt = torch.empty(E, dtype=torch.int32, device=dev)
+    rtok = torch.empty(R, dtype=torch.int32, device=dev)
+    in_rank = torch.empty(T, R, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        res = ep.ep_layout(idx, E, R, w.align, w.capacity, num_tokens_per_expert=cnt,
+                           num_tokens_per_rank=rtok, is_token_in_rank=in_rank)
+        if ev is not None:
+            ev[1].record(stream)
+        ep.ep_dispatch(res.handle, x, w.fp8, recv, scales)
+        if ev is not None:
+            ev[2].record(stream)
+        ep.ep_combine(res.handle, y, tw, out)
+        if ev is not None:
+            ev[3].record(stream)
+        return res.handle
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step().free()
+    torch.cuda.synchronize()
+    assert step().check() == ep.EP_OK
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    handles = []
+    for i in range(args.steps):
+        flush.zero_()
+        handles.append(step(events[i]))
+        if len(handles) > 4:
+            handles.pop(0).free()
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    status = handles[-1].check()
+    for h in handles:
+        h.free()
+    if status != ep.EP_OK:
+        raise SystemExit("device error: %s" % ep.status_str(status))
+
+    lay = [e[0].elapsed_time(e[1]) for e in events]
+    dis = [e[1].elapsed_time(e[2]) for e in events]
+    com = [e[2].elapsed_time(e[3]) for e in events]
+    stp = [e[0].elapsed_time(e[3]) for e in events]
+    mean = lambda v: sum(v) / len(v)  # noqa: E731
+    step_ms = reduce_max(mean(stp), world)
+    lay_ms, dis_ms, com_ms = (reduce_max(mean(v), world) for v in (lay, dis, com))
+    total_bytes = reduce_sum(nbytes["step"] * args.steps, world)
+    value = total_bytes / (step_ms * args.steps / 1e3) / 1e9
+
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"]
+    kern = {
+        "layout": {"us": lay_ms * 1e3, "bytes": nbytes["layout"], "launches_per_step": 3},
+        "dispatch": {"us": dis_ms * 1e3, "bytes": nbytes["dispatch"],
+                     "gbs": nbytes["dispatch"] / (dis_ms / 1e3) / 1e9},
+        "combine": {"us": com_ms * 1e3, "bytes": nbytes["combine"],
+                    "gbs": nbytes["combine"] / (com_ms / 1e3) / 1e9},
+    }
+    for kname in ("dispatch", "combine"):
+        kern[kname]["frac_of_peak"] = kern[kname]["gbs"] / peak
+        kern[kname]["frac_of_8tbs_nominal"] = kern[kname]["gbs"] / 8000.0
+    dom = "combine" if com_ms >= dis_ms else "dispatch"
+    src_file = {"combine": "combine.cu", "dispatch": "dispatch.cu"}[dom]
+    tr = NCU_TRAFFIC.get((w.name, dom))
+    traffic = tr["bytes"] if tr and tr["sha"] == source_sha(src_file) else None
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["gbs"], "peak": peak,
+                "unit": "GB/s", "frac": kern[dom]["gbs"] / peak, "traffic": traffic,
+                "algorithmic_bytes": nbytes[dom], "peak_source": peaks["source"]}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y, nbytes, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, seed)
+
+    if rank == 0:
+        line = {
+            "metric": "dispatch/combine HBM GB/s & % of peak; us/call at 8192 tok, H=7168, top-8",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(w, world),
+            "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 5 * args.steps, "clocks": clocks, "wall_s": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y_dev, nbytes, world):
+    """Same step through the public API from pinned host buffers: H2D of x,
+    topk_idx, topk_w and the expert outputs y, the three calls, D2H of out."""
+    T, H, E, R = w.T, w.H, w.E, w.R
+    xh = x_cpu.pin_memory()
+    ih = idx_cpu.pin_memory()
+    th = tw_cpu.pin_memory()
+    yh = y_dev.cpu().pin_memory()
+    oh = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(xh, device=dev)
+    idd = torch.empty_like(ih, device=dev)
+    twd = torch.empty_like(th, device=dev)
+    yd = torch.empty_like(yh, device=dev)
+    rdt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
+    rows = yd.shape[0]
+    recv = torch.empty(rows, H, dtype=rdt, device=dev)
+    scales = torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if w.fp8 else None
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in (xh, ih, th, yh))
+    d2h = oh.numel() * oh.element_size()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        xd.copy_(xh, non_blocking=True)
+        idd.copy_(ih, non_blocking=True)
+        twd.copy_(th, non_blocking=True)
+        yd.copy_(yh, non_blocking=True)
+        res = ep.ep_layout(idd, E, R, w.align, w.capacity)
+        ep.ep_dispatch(res.handle, xd, w.fp8, recv, scales)
+        ep.ep_combine(res.handle, yd, twd, out)
+        oh.copy_(out, non_blocking=True)
+        return res.handle
+
+    n_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step().free()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    handles = []
+    e0.record(stream)
+    for _ in range(n_steps):
+        handles.append(step())
+    e1.record(stream)
+    torch.cuda.synchronize()
+    for h in handles:
+        h.free()
+    ms = reduce_max(e0.elapsed_time(e1) / n_steps, world)
+    total = reduce_sum(nbytes["step"], world)
+    return {"value": total / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps}
+
+
+def main():
+    args = parse()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,111 @@
+// combine.cu -- top-k weighted reduction of expert outputs back to source
+// token order, in BF16.
+//
+// Combine as the pages describe it ("DeepEP (DeepEveryParallel)
+// Documentation", items 3 and 10: expert outputs are reduced back to the
+// tokens they came from; BF16 combine in "DeepSeek publica DeepEP ...",
+// news.hada.io, "Resultados de medición de rendimiento").  This library
+// fixes the arithmetic: for every token t and channel i,
+//     acc = +0.0f;  for j = 0..k-1 with pos[t][j] >= 0:
+//         acc = fmaf(w[t][j], y[pos[t][j]][i], acc);
+//     out[t][i] = bf16 round-to-nearest-even(acc).
+// A gather of k rows per token plus FMAs: HBM bound (k*H*2 bytes read and H*2
+// written per token).  Each thread owns one 16-byte vector (8 channels) of
+// one token, issues all k row loads of a batch before it accumulates (k
+// independent 16-byte loads in flight per thread, read-only non-coherent path
+// without L1 allocation: y is never written during the kernel), then runs the
+// FMA chain in slot order and stores 16 bytes.
+#include <cuda_bf16.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kCombineThreads = 128;
+constexpr int kLoadBatch = 8;  // row loads issued back to back before accumulating
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4 &v) {
+    acc[0] = __fmaf_rn(w, __uint_as_float(v.x << 16), acc[0]);
+    acc[1] = __fmaf_rn(w, __uint_as_float(v.x & 0xffff0000u), acc[1]);
+    acc[2] = __fmaf_rn(w, __uint_as_float(v.y << 16), acc[2]);
+    acc[3] = __fmaf_rn(w, __uint_as_float(v.y & 0xffff0000u), acc[3]);
+    acc[4] = __fmaf_rn(w, __uint_as_float(v.z << 16), acc[4]);
+    acc[5] = __fmaf_rn(w, __uint_as_float(v.z & 0xffff0000u), acc[5]);
+    acc[6] = __fmaf_rn(w, __uint_as_float(v.w << 16), acc[6]);
+    acc[7] = __fmaf_rn(w, __uint_as_float(v.w & 0xffff0000u), acc[7]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return l | (h << 16);
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
+    __shared__ int32_t p_s[kMaxTopk];
+    __shared__ float w_s[kMaxTopk];
+    const int t = blockIdx.x / a.blocks_per_token;
+    const int cb = blockIdx.x - t * a.blocks_per_token;
+    if (threadIdx.x < a.k) {
+        p_s[threadIdx.x] = __ldg(a.pos + (int64_t)t * a.k + threadIdx.x);
+        w_s[threadIdx.x] = __ldg(a.w + (int64_t)t * a.k + threadIdx.x);
+    }
+    __syncthreads();
+
+    const size_t row_bytes = (size_t)a.H * 2;
+#pragma unroll
+    for (int vi = 0; vi < VPT; ++vi) {
+        const int v = (cb * VPT + vi) * kCombineThreads + threadIdx.x;
+        if (v >= a.nvec) break;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j0 = 0; j0 < a.k; j0 += kLoadBatch) {
+            uint4 r[kLoadBatch];
+#pragma unroll
+            for (int jj = 0; jj < kLoadBatch; ++jj) {
+                const int j = j0 + jj;
+                const int p = (j < a.k) ? p_s[j] : -1;
+                if (p >= 0) r[jj] = ld_stream_v4(a.y + (size_t)p * row_bytes + (size_t)v * 16);
+            }
+#pragma unroll
+            for (int jj = 0; jj < kLoadBatch; ++jj) {
+                const int j = j0 + jj;
+                const int p = (j < a.k) ? p_s[j] : -1;
+                if (p >= 0) fma8(acc, w_s[j], r[jj]);
+            }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4 *>(a.out + (size_t)t * row_bytes + (size_t)v * 16) = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
+    if (a.T == 0) return cudaSuccess;
+    const long long blocks = (long long)a.T * a.blocks_per_token;
+    if ((long long)a.blocks_per_token * a.vpt * kCombineThreads < a.nvec)
+        return cudaErrorInvalidConfiguration;
+    switch (a.vpt) {
+        case 1: combine_kernel<1><<<(unsigned)blocks, kCombineThreads, 0, s>>>(a); break;
+        case 2: combine_kernel<2><<<(unsigned)blocks, kCombineThreads, 0, s>>>(a); break;
+        case 4: combine_kernel<4><<<(unsigned)blocks, kCombineThreads, 0, s>>>(a); break;
+        default: return cudaErrorInvalidConfiguration;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ep

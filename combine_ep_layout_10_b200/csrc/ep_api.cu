@@ -1,0 +1,312 @@
+// ep_api.cu -- the C ABI declared in include/ep.h: argument validation,
+// handle ownership and kernel launches.  Every step of the data path runs in
+// the kernels of layout.cu, dispatch.cu and combine.cu; nothing here touches
+// tensor data on the host.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceInfo g_info[kMaxDevices];
+bool g_have[kMaxDevices];
+
+constexpr int kDefaultTileTokens = 128;
+constexpr int kMaxTiles = 512;
+constexpr int kMaxChunkChannels = 8192;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+ep_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return EP_OK;
+    if (e == cudaErrorMemoryAllocation) return EP_ERR_OOM;
+    if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver || e == cudaErrorNoKernelImageForDevice)
+        return EP_ERR_NO_DEVICE;
+    return EP_ERR_CUDA;
+}
+
+// The current device, checked to be a Blackwell sm_100 part.
+ep_status current_device(int *dev, DeviceInfo *info) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    if ((e = device_info(*dev, info)) != cudaSuccess) return cuda_status(e);
+    if (info->cc_major != 10) return EP_ERR_NO_DEVICE;
+    return EP_OK;
+}
+
+}  // namespace
+
+cudaError_t device_info(int device, DeviceInfo *out) {
+    if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_have[device]) {
+        DeviceInfo d{};
+        cudaError_t e;
+        if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, device)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, device)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                        device)) != cudaSuccess)
+            return e;
+        g_info[device] = d;
+        g_have[device] = true;
+    }
+    *out = g_info[device];
+    return cudaSuccess;
+}
+
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" {
+
+const char *ep_status_str(ep_status s) {
+    switch (s) {
+        case EP_OK: return "EP_OK";
+        case EP_ERR_INVALID_ARG: return "EP_ERR_INVALID_ARG";
+        case EP_ERR_BAD_EXPERT_ID: return "EP_ERR_BAD_EXPERT_ID";
+        case EP_ERR_CAPACITY: return "EP_ERR_CAPACITY";
+        case EP_ERR_CUDA: return "EP_ERR_CUDA";
+        case EP_ERR_OOM: return "EP_ERR_OOM";
+        case EP_ERR_TIMEOUT: return "EP_ERR_TIMEOUT";
+        case EP_ERR_NO_DEVICE: return "EP_ERR_NO_DEVICE";
+    }
+    return "EP_ERR_UNKNOWN";
+}
+
+size_t ep_max_recv_rows(int T, int k, int E, int A, int C) {
+    if (T < 0 || k < 1 || k > kMaxTopk || E < 1 || E > kMaxExperts || A < 1 || C < 0) return 0;
+    if (C > 0) return (size_t)E * (size_t)C;
+    return (size_t)T * (size_t)k + (size_t)E * (size_t)(A - 1);
+}
+
+ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, int C,
+                    int32_t *out_cnt, int32_t *out_rank_tok, uint8_t *out_in_rank,
+                    ep_handle **out_handle, ep_stream_t stream) {
+    if (out_handle == nullptr) return EP_ERR_INVALID_ARG;
+    *out_handle = nullptr;
+    if (T < 0 || k < 1 || k > kMaxTopk || E < 1 || E > kMaxExperts || R < 1 || R > E || E % R != 0 ||
+        A < 1 || C < 0 || (C > 0 && C % A != 0))
+        return EP_ERR_INVALID_ARG;
+    if ((int64_t)T * k >= (int64_t)1 << 31) return EP_ERR_INVALID_ARG;
+    const size_t n_rows = ep_max_recv_rows(T, k, E, A, C);
+    if (n_rows >= ((size_t)1 << 31)) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (topk_idx == nullptr || !aligned(topk_idx, 4))) return EP_ERR_INVALID_ARG;
+    if ((out_cnt && !aligned(out_cnt, 4)) || (out_rank_tok && !aligned(out_rank_tok, 4)))
+        return EP_ERR_INVALID_ARG;
+
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+
+    int tile_tokens = kDefaultTileTokens;
+    if ((T + tile_tokens - 1) / tile_tokens > kMaxTiles)
+        tile_tokens = (int)round_up((size_t)((T + kMaxTiles - 1) / kMaxTiles), 32);
+    const int ntiles = (T + tile_tokens - 1) / tile_tokens;
+
+    // One stream-ordered allocation, every array 256-byte aligned.
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    };
+    const size_t o_err = carve(4);
+    const size_t o_pos = carve((size_t)T * k * 4);
+    const size_t o_src = carve(n_rows * 4);
+    const size_t o_seg = carve((size_t)(E + 1) * 4);
+    const size_t o_roff = carve((size_t)(R + 1) * 4);
+    const size_t o_cnt = carve((size_t)E * 4);
+    const size_t o_tcnt = carve((size_t)ntiles * E * 4);
+    const size_t o_trank = carve((size_t)ntiles * R * 4);
+    void *block = nullptr;
+    cudaError_t e = cudaMallocAsync(&block, off, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    ep_handle *h = new (std::nothrow) ep_handle;
+    if (h == nullptr) {
+        cudaFreeAsync(block, stream);
+        return EP_ERR_OOM;
+    }
+    unsigned char *b = static_cast<unsigned char *>(block);
+    h->T = T; h->k = k; h->E = E; h->R = R; h->align = A; h->capacity = C;
+    h->experts_per_rank = E / R;
+    h->tile_tokens = tile_tokens;
+    h->ntiles = ntiles;
+    h->n_rows = (int64_t)n_rows;
+    h->device = dev;
+    h->stream = stream;
+    h->block = block;
+    h->err = reinterpret_cast<uint32_t *>(b + o_err);
+    h->pos = reinterpret_cast<int32_t *>(b + o_pos);
+    h->src_idx = reinterpret_cast<int32_t *>(b + o_src);
+    h->seg = reinterpret_cast<int32_t *>(b + o_seg);
+    h->rank_off = reinterpret_cast<int32_t *>(b + o_roff);
+    h->cnt = reinterpret_cast<int32_t *>(b + o_cnt);
+    h->tile_cnt = reinterpret_cast<int32_t *>(b + o_tcnt);
+    h->tile_rank = reinterpret_cast<int32_t *>(b + o_trank);
+
+    LayoutArgs a{};
+    a.topk_idx = topk_idx;
+    a.T = T; a.k = k; a.E = E; a.R = R; a.epr = E / R; a.align = A; a.capacity = C;
+    a.tile_tokens = tile_tokens;
+    a.ntiles = ntiles;
+    a.sub_tokens = std::max(1, std::min(tile_tokens, 4096 / R));
+    a.scan_parts_e = std::max(1, std::min(std::max(ntiles, 1), 1024 / E));
+    a.scan_parts_r = std::max(1, std::min(std::max(ntiles, 1), 1024 / R));
+    a.pos_warps = std::min(8, std::max(1, 12288 / E));
+    a.n_rows = (int64_t)n_rows;
+    a.pos = h->pos; a.src_idx = h->src_idx; a.seg = h->seg; a.rank_off = h->rank_off;
+    a.cnt = h->cnt; a.tile_cnt = h->tile_cnt; a.tile_rank = h->tile_rank; a.err = h->err;
+    a.out_cnt = out_cnt;
+    a.out_rank_tok = out_rank_tok;
+    a.out_in_rank = out_in_rank;
+
+    e = cudaMemsetAsync(h->err, 0, 4, stream);
+    if (e == cudaSuccess) e = launch_layout(a, stream);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(block, stream);
+        delete h;
+        return cuda_status(e);
+    }
+    *out_handle = h;
+    return EP_OK;
+}
+
+ep_status ep_dispatch(const ep_handle *h, const void *x, int H, int use_fp8, void *recv_x,
+                      float *recv_scales, int32_t *recv_src_idx, size_t recv_rows,
+                      ep_stream_t stream) {
+    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (use_fp8 && H % 128 != 0) return EP_ERR_INVALID_ARG;
+    if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    if (h->T > 0) {
+        if (x == nullptr || recv_x == nullptr || !aligned(x, 16) || !aligned(recv_x, 16))
+            return EP_ERR_INVALID_ARG;
+        if (use_fp8 && (recv_scales == nullptr || !aligned(recv_scales, 4))) return EP_ERR_INVALID_ARG;
+    }
+    if (recv_src_idx != nullptr && !aligned(recv_src_idx, 4)) return EP_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != h->device) return EP_ERR_INVALID_ARG;
+
+    const int align_ch = use_fp8 ? 128 : 8;
+    const int nchunks = (H + kMaxChunkChannels - 1) / kMaxChunkChannels;
+    const int chunk = (int)round_up((size_t)((H + nchunks - 1) / nchunks), align_ch);
+
+    DispatchArgs a{};
+    a.x = static_cast<const uint8_t *>(x);
+    a.pos = h->pos;
+    a.recv = static_cast<uint8_t *>(recv_x);
+    a.scales = recv_scales;
+    a.err = h->err;
+    a.T = h->T; a.k = h->k; a.H = H;
+    a.chunk = chunk;
+    a.nchunks = (H + chunk - 1) / chunk;
+    a.nunits = (long long)h->T * a.nchunks;
+    a.stages = use_fp8 ? 3 : 4;
+    cudaError_t e = launch_dispatch(a, use_fp8 != 0, info.num_sms, stream);
+    if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)
+        e = cudaMemcpyAsync(recv_src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
+    return cuda_status(e);
+}
+
+ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int H, size_t recv_rows,
+                     void *out, ep_stream_t stream) {
+    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    if (h->T > 0) {
+        if (y == nullptr || out == nullptr || topk_w == nullptr) return EP_ERR_INVALID_ARG;
+        if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_w, 4)) return EP_ERR_INVALID_ARG;
+    }
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != h->device) return EP_ERR_INVALID_ARG;
+
+    CombineArgs a{};
+    a.y = static_cast<const uint8_t *>(y);
+    a.w = topk_w;
+    a.pos = h->pos;
+    a.out = static_cast<uint8_t *>(out);
+    a.T = h->T; a.k = h->k; a.H = H;
+    a.nvec = H / 8;
+    a.vpt = 1;
+    a.blocks_per_token = (a.nvec + 127) / 128;
+    return cuda_status(launch_combine(a, stream));
+}
+
+void ep_handle_free(ep_handle *h) {
+    if (h == nullptr) return;
+    if (h->block != nullptr) {
+        if (cudaFreeAsync(h->block, h->stream) != cudaSuccess) {
+            (void)cudaGetLastError();
+            cudaFree(h->block);
+        }
+    }
+    delete h;
+}
+
+ep_status ep_handle_get_info(const ep_handle *h, ep_handle_info *info) {
+    if (h == nullptr || info == nullptr) return EP_ERR_INVALID_ARG;
+    info->num_tokens = h->T;
+    info->num_topk = h->k;
+    info->num_experts = h->E;
+    info->num_ranks = h->R;
+    info->expert_alignment = h->align;
+    info->capacity = h->capacity;
+    info->num_recv_rows = (size_t)h->n_rows;
+    return EP_OK;
+}
+
+ep_status ep_handle_export(const ep_handle *h, int32_t *pos, int32_t *src_idx, int32_t *seg,
+                           int32_t *rank_off, ep_stream_t stream) {
+    if (h == nullptr) return EP_ERR_INVALID_ARG;
+    cudaError_t e = cudaSuccess;
+    if (pos && h->T > 0)
+        e = cudaMemcpyAsync(pos, h->pos, (size_t)h->T * h->k * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess && src_idx && h->n_rows > 0)
+        e = cudaMemcpyAsync(src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess && seg)
+        e = cudaMemcpyAsync(seg, h->seg, (size_t)(h->E + 1) * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess && rank_off)
+        e = cudaMemcpyAsync(rank_off, h->rank_off, (size_t)(h->R + 1) * 4, cudaMemcpyDeviceToDevice, stream);
+    return cuda_status(e);
+}
+
+ep_status ep_handle_counts_host(const ep_handle *h, int32_t *host_counts, ep_stream_t stream) {
+    if (h == nullptr || host_counts == nullptr) return EP_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemcpyAsync(host_counts, h->cnt, (size_t)h->E * 4, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    return cuda_status(e);
+}
+
+ep_status ep_handle_check(const ep_handle *h, ep_stream_t stream) {
+    if (h == nullptr) return EP_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, h->err, 4, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (word & kErrBadExpertId) return EP_ERR_BAD_EXPERT_ID;
+    if (word & kErrCapacity) return EP_ERR_CAPACITY;
+    if (word & kErrTimeout) return EP_ERR_TIMEOUT;
+    return EP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,252 @@
+"""Python binding of the C ABI in include/ep.h (libep_b200.so).
+
+Argument marshalling only: every step of layout, dispatch and combine runs in
+the library's CUDA kernels.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the CUDA library is missing or the device is
+not an sm_100 part, the calls raise.
+
+The names follow the C ABI: ep_max_recv_rows, ep_layout, ep_dispatch,
+ep_combine, ep_handle_free (plus the handle accessors).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libep_b200.so")
+
+EP_OK = 0
+EP_ERR_INVALID_ARG = 1
+EP_ERR_BAD_EXPERT_ID = 2
+EP_ERR_CAPACITY = 3
+EP_ERR_CUDA = 4
+EP_ERR_OOM = 5
+EP_ERR_TIMEOUT = 6
+EP_ERR_NO_DEVICE = 7
+
+#: Every symbol the ABI exports (include/ep.h).
+ABI_SYMBOLS = (
+    "ep_status_str", "ep_max_recv_rows", "ep_layout", "ep_dispatch", "ep_combine",
+    "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
+    "ep_handle_check",
+)
+
+
+class EpError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s: %s" % (what, status_str(status)))
+        self.status = status
+
+
+class _HandleInfo(ctypes.Structure):
+    _fields_ = [("num_tokens", ctypes.c_int), ("num_topk", ctypes.c_int),
+                ("num_experts", ctypes.c_int), ("num_ranks", ctypes.c_int),
+                ("expert_alignment", ctypes.c_int), ("capacity", ctypes.c_int),
+                ("num_recv_rows", ctypes.c_size_t)]
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libep_b200.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libep_b200.so is missing (%s); build it with "
+                               "`python -m combine_ep_layout_10_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.ep_status_str.argtypes = [I]
+        L.ep_status_str.restype = ctypes.c_char_p
+        L.ep_max_recv_rows.argtypes = [I, I, I, I, I]
+        L.ep_max_recv_rows.restype = S
+        L.ep_layout.argtypes = [P, I, I, I, I, I, I, P, P, P, ctypes.POINTER(P), P]
+        L.ep_layout.restype = I
+        L.ep_dispatch.argtypes = [P, P, I, I, P, P, P, S, P]
+        L.ep_dispatch.restype = I
+        L.ep_combine.argtypes = [P, P, P, I, S, P, P]
+        L.ep_combine.restype = I
+        L.ep_handle_free.argtypes = [P]
+        L.ep_handle_free.restype = None
+        L.ep_handle_get_info.argtypes = [P, ctypes.POINTER(_HandleInfo)]
+        L.ep_handle_get_info.restype = I
+        L.ep_handle_export.argtypes = [P, P, P, P, P, P]
+        L.ep_handle_export.restype = I
+        L.ep_handle_counts_host.argtypes = [P, P, P]
+        L.ep_handle_counts_host.restype = I
+        L.ep_handle_check.argtypes = [P, P]
+        L.ep_handle_check.restype = I
+        _LIB = L
+    return _LIB
+
+
+def status_str(status: int) -> str:
+    return lib().ep_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != EP_OK:
+        raise EpError(status, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev_ptr(t: Optional[torch.Tensor], dtype, name: str, shape=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def ep_max_recv_rows(num_tokens: int, num_topk: int, num_experts: int,
+                     expert_alignment: int = 1, capacity: int = 0) -> int:
+    return int(lib().ep_max_recv_rows(num_tokens, num_topk, num_experts, expert_alignment, capacity))
+
+
+class Handle:
+    """Owner of an ep_handle* (the pages' EPHandle).  Reusable across calls
+    while the routing is unchanged (the cached-handle decoding path)."""
+
+    def __init__(self, ptr: ctypes.c_void_p, device: torch.device):
+        self._ptr = ptr
+        self.device = device
+        info = _HandleInfo()
+        _check(lib().ep_handle_get_info(ptr, ctypes.byref(info)), "ep_handle_get_info")
+        self.num_tokens = info.num_tokens
+        self.num_topk = info.num_topk
+        self.num_experts = info.num_experts
+        self.num_ranks = info.num_ranks
+        self.expert_alignment = info.expert_alignment
+        self.capacity = info.capacity
+        self.num_recv_rows = int(info.num_recv_rows)
+
+    @property
+    def ptr(self) -> ctypes.c_void_p:
+        if self._ptr is None:
+            raise RuntimeError("handle already freed")
+        return self._ptr
+
+    def export(self, stream=None) -> dict:
+        """Device copies of pos [T,k], src_idx [rows], seg [E+1], rank_off [R+1]."""
+        dev = self.device
+        pos = torch.empty(self.num_tokens, self.num_topk, dtype=torch.int32, device=dev)
+        src = torch.empty(self.num_recv_rows, dtype=torch.int32, device=dev)
+        seg = torch.empty(self.num_experts + 1, dtype=torch.int32, device=dev)
+        roff = torch.empty(self.num_ranks + 1, dtype=torch.int32, device=dev)
+        _check(lib().ep_handle_export(self.ptr, _dev_ptr(pos, None, "pos"), _dev_ptr(src, None, "src"),
+                                      _dev_ptr(seg, None, "seg"), _dev_ptr(roff, None, "rank_off"),
+                                      _stream(stream)), "ep_handle_export")
+        return {"pos": pos, "src_idx": src, "seg": seg, "rank_off": roff}
+
+    def counts_host(self, stream=None) -> list:
+        """num_recv_tokens_per_expert_list (synchronises the stream)."""
+        buf = (ctypes.c_int32 * self.num_experts)()
+        _check(lib().ep_handle_counts_host(self.ptr, buf, _stream(stream)), "ep_handle_counts_host")
+        return list(buf)
+
+    def check(self, stream=None) -> int:
+        """The device error word as a status (synchronises the stream)."""
+        return int(lib().ep_handle_check(self.ptr, _stream(stream)))
+
+    def free(self) -> None:
+        if self._ptr is not None:
+            lib().ep_handle_free(self._ptr)
+            self._ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+@dataclass
+class LayoutResult:
+    num_tokens_per_expert: torch.Tensor   # int32 [E]
+    num_tokens_per_rank: torch.Tensor     # int32 [R]
+    is_token_in_rank: torch.Tensor        # uint8 [T, R]
+    handle: Handle
+
+
+def ep_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, expert_alignment: int = 1,
+              capacity: int = 0, *, num_tokens_per_expert: Optional[torch.Tensor] = None,
+              num_tokens_per_rank: Optional[torch.Tensor] = None,
+              is_token_in_rank: Optional[torch.Tensor] = None, stream=None) -> LayoutResult:
+    if topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be [T, k]")
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if num_tokens_per_expert is None:
+        num_tokens_per_expert = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    if num_tokens_per_rank is None:
+        num_tokens_per_rank = torch.empty(num_ranks, dtype=torch.int32, device=dev)
+    if is_token_in_rank is None:
+        is_token_in_rank = torch.empty(T, num_ranks, dtype=torch.uint8, device=dev)
+    h = ctypes.c_void_p()
+    st = lib().ep_layout(_dev_ptr(topk_idx, torch.int32, "topk_idx"), T, k, num_experts, num_ranks,
+                         expert_alignment, capacity,
+                         _dev_ptr(num_tokens_per_expert, torch.int32, "num_tokens_per_expert", (num_experts,)),
+                         _dev_ptr(num_tokens_per_rank, torch.int32, "num_tokens_per_rank", (num_ranks,)),
+                         _dev_ptr(is_token_in_rank, torch.uint8, "is_token_in_rank", (T, num_ranks)),
+                         ctypes.byref(h), _stream(stream))
+    _check(st, "ep_layout")
+    return LayoutResult(num_tokens_per_expert, num_tokens_per_rank, is_token_in_rank, Handle(h, dev))
+
+
+def ep_dispatch(handle: Handle, x: torch.Tensor, use_fp8: bool, recv_x: Optional[torch.Tensor] = None,
+                recv_scales: Optional[torch.Tensor] = None, recv_src_idx: Optional[torch.Tensor] = None,
+                stream=None):
+    """Returns (recv_x, recv_scales or None, recv_src_idx or None)."""
+    T, H = x.shape
+    if T != handle.num_tokens:
+        raise ValueError("x has %d tokens, the handle %d" % (T, handle.num_tokens))
+    rows = handle.num_recv_rows
+    dt = torch.float8_e4m3fn if use_fp8 else torch.bfloat16
+    if recv_x is None:
+        recv_x = torch.empty(rows, H, dtype=dt, device=x.device)
+    if use_fp8 and recv_scales is None:
+        recv_scales = torch.empty(rows, H // 128, dtype=torch.float32, device=x.device)
+    if recv_x.dim() != 2 or recv_x.shape[1] != H:
+        raise ValueError("recv_x must be [rows, %d]" % H)
+    st = lib().ep_dispatch(handle.ptr, _dev_ptr(x, torch.bfloat16, "x"), H, 1 if use_fp8 else 0,
+                           _dev_ptr(recv_x, dt, "recv_x"),
+                           _dev_ptr(recv_scales, torch.float32, "recv_scales") if use_fp8 else None,
+                           _dev_ptr(recv_src_idx, torch.int32, "recv_src_idx"),
+                           recv_x.shape[0], _stream(stream))
+    _check(st, "ep_dispatch")
+    return recv_x, (recv_scales if use_fp8 else None), recv_src_idx
+
+
+def ep_combine(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    rows, H = y.shape
+    if out is None:
+        out = torch.empty(handle.num_tokens, H, dtype=torch.bfloat16, device=y.device)
+    st = lib().ep_combine(handle.ptr, _dev_ptr(y, torch.bfloat16, "y"),
+                          _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                   (handle.num_tokens, handle.num_topk)),
+                          H, rows, _dev_ptr(out, torch.bfloat16, "out", (handle.num_tokens, H)),
+                          _stream(stream))
+    _check(st, "ep_combine")
+    return out
+
+
+def ep_handle_free(handle: Handle) -> None:
+    handle.free()

@@ -1,0 +1,181 @@
+/*
+ * ep.h -- C ABI of the B200 (sm_100a) MoE expert-parallel layout / dispatch /
+ * combine library (libep_b200.so).
+ *
+ * The operations follow the interface the DeepEP pages describe:
+ *   - "DeepEP (DeepEveryParallel) Documentation" (docsearch.algolia.com),
+ *     item 10 "Perform MoE Dispatch and Combine for Training or Prefilling":
+ *     dispatch takes the hidden states, the top-k expert ids and weights, the
+ *     number of experts and the expert alignment, routes every token to its
+ *     experts and returns the received rows plus a handle with the routing
+ *     metadata; combine takes expert outputs and that handle and reduces them
+ *     back to the source tokens.
+ *   - the same page, item 3 "Perform MoE Dispatch and Combine for Inference
+ *     Decoding": a cached handle is passed again when the gating decision has
+ *     not changed, so the layout and its host synchronisation are skipped.
+ *   - "DeepSeek publica DeepEP, una biblioteca open source para entrenamiento
+ *     e inferencia MoE" (news.hada.io), section "Patrones de uso en
+ *     entrenamiento, prefill y decoding": the handle carries the per-expert
+ *     received-token counts the expert GEMMs need; section "Resultados de
+ *     medición de rendimiento": FP8 dispatch, BF16 combine.
+ *
+ * On one GPU the expert-parallel ranks are virtual: rank r owns experts
+ * [r*E/R, (r+1)*E/R) and the contiguous slice of receive rows of those
+ * experts.  Nothing crosses devices.
+ *
+ * Notation: T tokens, H hidden size, k top-k slots per token, E experts,
+ * R virtual ranks.  A slot is a pair (t, j), 0 <= j < k.
+ *
+ * Definition of the layout (the pages do not spell it out; this library
+ * fixes it so that results are bit-exact and independent of scheduling):
+ *   receive rows are expert-major; inside an expert's segment rows follow
+ *   (source token, slot) order.  Packed mode (capacity == 0): segment e
+ *   starts at seg[e] = sum over e' < e of align_up(cnt[e'], expert_alignment).
+ *   Padded mode (capacity > 0): segment e is rows [e*capacity, (e+1)*capacity).
+ *   A slot whose id is -1 is unused: no row, no combine term.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device (or managed) memory of the
+ *     current device; the caller allocates and owns them.  Pointers marked
+ *     "host" are ordinary host memory.
+ *   - Row-major, densely packed arrays.  x, recv_x, y and combined_x must be
+ *     16-byte aligned; recv_scales, topk_weights 4-byte aligned.
+ *   - All device work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and is asynchronous, unless a call says it
+ *     synchronises.
+ *   - Argument errors are detected on the host and returned at once with
+ *     nothing enqueued.  Data errors found on the device (an id outside
+ *     [-1, E), a padded expert over capacity, a timed-out wait) set the
+ *     handle's device error word instead; the outputs of that call are then
+ *     unspecified but every device write stays inside the buffers described
+ *     here.  ep_handle_check() reports the word.  No call traps, aborts or
+ *     throws across the ABI.
+ *   - Limits: 1 <= k <= 32, 1 <= E <= 4096, 1 <= R <= E, E % R == 0,
+ *     T * k < 2^31, H % 8 == 0 (bf16) and H % 128 == 0 (FP8).
+ */
+#ifndef EP_B200_EP_H
+#define EP_B200_EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that the header needs no CUDA include. */
+typedef struct CUstream_st *ep_stream_t;
+
+/* Opaque routing handle (the pages' EPHandle): owns device copies of the
+ * slot positions, the source-token index of every receive row, the expert
+ * segments, the rank slices, the per-expert counts and a device error word. */
+typedef struct ep_handle ep_handle;
+
+typedef enum ep_status {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1,   /* bad size, null or misaligned pointer, limits exceeded */
+    EP_ERR_BAD_EXPERT_ID = 2, /* a top-k id outside [-1, E) (device-detected) */
+    EP_ERR_CAPACITY = 3,      /* padded mode: an expert received more than `capacity` tokens */
+    EP_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+    EP_ERR_OOM = 5,           /* device allocation failed */
+    EP_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up */
+    EP_ERR_NO_DEVICE = 7      /* no CUDA device, or the device is not sm_100 */
+} ep_status;
+
+/* Human-readable name of a status.  Never NULL; static storage. */
+const char *ep_status_str(ep_status status);
+
+/* Upper bound on the receive rows a layout with these parameters can use:
+ * E * capacity in padded mode, T*k + E*(expert_alignment-1) in packed mode.
+ * recv_x / y must have at least this many rows.  Host only, pure.  Returns 0
+ * for invalid arguments. */
+size_t ep_max_recv_rows(int num_tokens, int num_topk, int num_experts,
+                        int expert_alignment, int capacity);
+
+/* Routing layout: the metadata part of the pages' dispatch (docsearch item
+ * 10; news.hada.io "Patrones de uso ...").  Computes, bit-exactly:
+ *   num_tokens_per_expert[e] = number of slots naming expert e       (device int32 [E], may be NULL)
+ *   num_tokens_per_rank[r]   = tokens with >= 1 expert on rank r      (device int32 [R], may be NULL)
+ *   is_token_in_rank[t][r]   = 1 if token t has an expert on rank r   (device uint8 [T, R], may be NULL)
+ * and a new handle holding pos[T][k] (receive row of each slot, -1 for
+ * unused or over-capacity slots), src_idx[rows] (source token of each
+ * receive row, -1 for padding), seg[E+1] and rank_off[R+1].
+ *   topk_idx: device int32 [T, k]; ids in [-1, E).
+ *   expert_alignment >= 1: packed segments are rounded up to a multiple of it.
+ *   capacity: 0 for packed mode, else rows per expert (a multiple of expert_alignment).
+ * On success *out_handle receives a handle that the caller frees with
+ * ep_handle_free().  The handle's device memory is allocated stream-ordered
+ * on `stream` (cudaMallocAsync).  T == 0 is allowed (empty handle). */
+ep_status ep_layout(const int32_t *topk_idx, int num_tokens, int num_topk,
+                    int num_experts, int num_ranks, int expert_alignment, int capacity,
+                    int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                    uint8_t *is_token_in_rank, ep_handle **out_handle, ep_stream_t stream);
+
+/* Dispatch (docsearch item 10, FP8 per "deepseek-ai/DeepEP" repolode
+ * "Funciones clave"): scatter every token's hidden row to the receive row of
+ * each of its valid slots.
+ *   x: device bf16 [T, H].
+ *   use_fp8 == 0: recv_x is device bf16 [recv_rows, H]; each row a bit copy of x[t].
+ *   use_fp8 != 0: recv_x is device e4m3 (OCP FP8 E4M3, 1 byte) [recv_rows, H] and
+ *     recv_scales device fp32 [recv_rows, H/128].  Per token and 128-channel
+ *     group g: amax = max |x|; scale = amax/448 (fp32, round to nearest);
+ *     codes = e4m3_rn_satfinite(x * (448/amax)) with 448/amax one rounded
+ *     fp32 division; an all-zero group gives scale 0 and codes 0x00.  The
+ *     same codes and scales go to all k rows of the token.
+ *   recv_src_idx: device int32 [recv_rows] or NULL; receives a copy of the
+ *     handle's src_idx (-1 on padding rows).
+ *   recv_rows: rows allocated in recv_x / recv_scales / recv_src_idx; must be
+ *     >= ep_max_recv_rows() of the handle's layout.
+ * Only rows that slots map to are written; padding rows keep their contents.
+ * No allocation, no host synchronisation: may be captured in a CUDA graph and
+ * reused with the same handle for every decoding step (docsearch item 3). */
+ep_status ep_dispatch(const ep_handle *handle, const void *x, int hidden, int use_fp8,
+                      void *recv_x, float *recv_scales, int32_t *recv_src_idx,
+                      size_t recv_rows, ep_stream_t stream);
+
+/* Combine (docsearch items 3 and 10; BF16 per news.hada.io "Resultados ..."):
+ *   combined_x[t][i] = bf16_rn( fma chain, j = 0..k-1 over slots with pos >= 0,
+ *                               acc = fmaf(topk_weights[t][j], y[pos[t][j]][i], acc),
+ *                               starting from acc = +0.0f )
+ *   y: device bf16 [recv_rows, H] (expert outputs, rows in the handle's layout).
+ *   topk_weights: device fp32 [T, k].
+ *   combined_x: device bf16 [T, H].  A token with no valid slot gets +0.0.
+ * No allocation, no host synchronisation; graph-capturable. */
+ep_status ep_combine(const ep_handle *handle, const void *y, const float *topk_weights,
+                     int hidden, size_t recv_rows, void *combined_x, ep_stream_t stream);
+
+/* Release a handle.  Its device memory is freed stream-ordered on the stream
+ * that created it (cudaFreeAsync); work that uses the handle on other streams
+ * must be ordered before that stream's current position by the caller.
+ * NULL is a no-op. */
+void ep_handle_free(ep_handle *handle);
+
+/* Handle geometry (host only, no device work). */
+typedef struct ep_handle_info {
+    int num_tokens, num_topk, num_experts, num_ranks, expert_alignment, capacity;
+    size_t num_recv_rows; /* = ep_max_recv_rows(...) of this layout */
+} ep_handle_info;
+ep_status ep_handle_get_info(const ep_handle *handle, ep_handle_info *info);
+
+/* Copy the handle's metadata into caller buffers (device-to-device, async on
+ * `stream`).  Any destination may be NULL.
+ *   pos: device int32 [T, k]; src_idx: device int32 [num_recv_rows];
+ *   seg: device int32 [E+1]; rank_off: device int32 [R+1]. */
+ep_status ep_handle_export(const ep_handle *handle, int32_t *pos, int32_t *src_idx,
+                           int32_t *seg, int32_t *rank_off, ep_stream_t stream);
+
+/* The pages' num_recv_tokens_per_expert_list: per-expert counts copied to
+ * host int32 [E].  Synchronises `stream`. */
+ep_status ep_handle_counts_host(const ep_handle *handle, int32_t *host_counts,
+                                ep_stream_t stream);
+
+/* Read the handle's device error word after the work enqueued on `stream`
+ * so far.  Synchronises `stream`.  Returns EP_OK, EP_ERR_BAD_EXPERT_ID,
+ * EP_ERR_CAPACITY or EP_ERR_TIMEOUT (the first set, in that order). */
+ep_status ep_handle_check(const ep_handle *handle, ep_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_EP_H */

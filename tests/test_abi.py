@@ -1,0 +1,85 @@
+"""The C-ABI library loads and exports every symbol include/ep.h declares;
+host-side argument validation works without a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from combine_ep_layout_10_b200 import build as B
+from combine_ep_layout_10_b200 import ep
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return ep.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ep.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ep_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(ep.ABI_SYMBOLS) == names
+
+
+def test_status_strings(L):
+    assert ep.status_str(0) == "EP_OK"
+    assert ep.status_str(3) == "EP_ERR_CAPACITY"
+    assert ep.status_str(99) == "EP_ERR_UNKNOWN"
+
+
+def test_max_recv_rows(L):
+    assert ep.ep_max_recv_rows(8192, 8, 256) == 65536
+    assert ep.ep_max_recv_rows(8192, 8, 256, 4) == 65536 + 256 * 3
+    assert ep.ep_max_recv_rows(128, 8, 256, 1, 128) == 32768
+    assert ep.ep_max_recv_rows(-1, 8, 256) == 0
+    assert ep.ep_max_recv_rows(16, 33, 256) == 0
+
+
+def _layout_status(L, T, k, E, R, A=1, C=0, idx=None):
+    h = ctypes.c_void_p()
+    return L.ep_layout(idx, T, k, E, R, A, C, None, None, None, ctypes.byref(h), None)
+
+
+def test_layout_argument_errors_on_host(L):
+    fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    assert _layout_status(L, 4, 2, 4, 3, idx=fake) == ep.EP_ERR_INVALID_ARG       # E % R
+    assert _layout_status(L, 4, 33, 64, 2, idx=fake) == ep.EP_ERR_INVALID_ARG     # k > 32
+    assert _layout_status(L, 4, 2, 8192, 2, idx=fake) == ep.EP_ERR_INVALID_ARG    # E > 4096
+    assert _layout_status(L, 4, 2, 4, 2, A=0, idx=fake) == ep.EP_ERR_INVALID_ARG  # align
+    assert _layout_status(L, 4, 2, 4, 2, A=2, C=3, idx=fake) == ep.EP_ERR_INVALID_ARG
+    assert _layout_status(L, 4, 2, 4, 2, idx=None) == ep.EP_ERR_INVALID_ARG       # null ids
+    assert _layout_status(L, 4, 2, 4, 2, idx=ctypes.c_void_p(258)) == ep.EP_ERR_INVALID_ARG  # misaligned
+    assert L.ep_layout(fake, 4, 2, 4, 2, 1, 0, None, None, None, None, None) == ep.EP_ERR_INVALID_ARG
+
+
+def test_dispatch_combine_argument_errors_on_host(L):
+    assert L.ep_dispatch(None, None, 128, 0, None, None, None, 0, None) == ep.EP_ERR_INVALID_ARG
+    assert L.ep_combine(None, None, None, 128, 0, None, None) == ep.EP_ERR_INVALID_ARG
+    L.ep_handle_free(None)  # no-op
+    info = ep._HandleInfo()
+    assert L.ep_handle_get_info(None, ctypes.byref(info)) == ep.EP_ERR_INVALID_ARG
+    assert L.ep_handle_check(None, None) == ep.EP_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_no_device_is_reported(L):
+    assert _layout_status(L, 0, 2, 4, 2) == ep.EP_ERR_NO_DEVICE
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(ep, "_LIB", None)
+    monkeypatch.setattr(ep, "LIB_PATH", "/nonexistent/libep_b200.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        ep.lib()
