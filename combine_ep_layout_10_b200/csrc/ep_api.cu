@@ -83,6 +83,7 @@ const char *ep_status_str(ep_status s) {
         case EP_ERR_OOM: return "EP_ERR_OOM";
         case EP_ERR_TIMEOUT: return "EP_ERR_TIMEOUT";
         case EP_ERR_NO_DEVICE: return "EP_ERR_NO_DEVICE";
+        case EP_ERR_SCRATCH_LIMIT: return "EP_ERR_SCRATCH_LIMIT";
     }
     return "EP_ERR_UNKNOWN";
 }

@@ -1,0 +1,134 @@
+// noalloc.cu -- ep_layout_noalloc: the routing layout without any device
+// allocation, for callers that cannot allocate.
+//
+// Who needs it: a serving loop whose device memory is planned once at start-up
+// by a static memory planner (every byte pre-carved, no allocator on the hot
+// path); code that runs under another framework's allocator and may not touch
+// the CUDA allocator behind its back; and latency-critical loops that must not
+// risk cudaMalloc's implicit device synchronisation.  Those callers pass every
+// input and output buffer themselves; the only other device memory this call
+// uses is the fixed scratch array below.
+//
+// The scratch (the layout's per-tile count matrices, a per-expert count
+// buffer and a fallback error word) is a file-scope __device__ array of
+// EP_NOALLOC_SCRATCH_WORDS 32-bit words: it is created when the library's
+// device code is loaded and every GPU that loads the library holds it until
+// the process exits.  Its device address is looked up once per device with
+// cudaGetSymbolAddress (host code cannot use the array's name as a device
+// pointer), by the first call on that device with that device current.  All
+// calls on a device share the array, so two calls whose work overlaps on the
+// GPU (different streams, no ordering between them) race on it; calls on one
+// stream are ordered and safe.  Nothing in it needs to start at zero: the
+// count kernel overwrites every tile entry it uses and the error word is
+// cleared by this call.
+#include <algorithm>
+#include <mutex>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+static __device__ __align__(256) int32_t g_layout_scratch[EP_NOALLOC_SCRATCH_WORDS];
+
+constexpr int kMaxDevicesNoAlloc = 64;
+std::mutex g_scratch_mu;
+int32_t *g_scratch_ptr[kMaxDevicesNoAlloc];
+
+bool is_aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+ep_status status_of(cudaError_t e) {
+    if (e == cudaSuccess) return EP_OK;
+    if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver || e == cudaErrorNoKernelImageForDevice)
+        return EP_ERR_NO_DEVICE;
+    return EP_ERR_CUDA;
+}
+
+// Device address of the scratch array on `dev` (which is current).
+ep_status scratch_for_device(int dev, int32_t **out) {
+    if (dev < 0 || dev >= kMaxDevicesNoAlloc) return EP_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_layout_scratch);
+        if (e != cudaSuccess || p == nullptr) return e != cudaSuccess ? status_of(e) : EP_ERR_CUDA;
+        g_scratch_ptr[dev] = static_cast<int32_t *>(p);
+    }
+    *out = g_scratch_ptr[dev];
+    return EP_OK;
+}
+
+}  // namespace
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, int E, int R, int A, int C,
+                                       int32_t *out_cnt, int32_t *out_rank_tok, uint8_t *out_in_rank,
+                                       int32_t *pos, int32_t *src_idx, int32_t *seg, int32_t *rank_off,
+                                       uint32_t *error_word, ep_stream_t stream) {
+    if (T < 0 || k < 1 || k > kMaxTopk || E < 1 || E > kMaxExperts || R < 1 || R > E || E % R != 0 ||
+        A < 1 || C < 0 || (C > 0 && C % A != 0))
+        return EP_ERR_INVALID_ARG;
+    if ((int64_t)T * k >= (int64_t)1 << 31) return EP_ERR_INVALID_ARG;
+    const size_t n_rows = ep_max_recv_rows(T, k, E, A, C);
+    if (n_rows >= ((size_t)1 << 31)) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (topk_idx == nullptr || !is_aligned(topk_idx, 4) || pos == nullptr || !is_aligned(pos, 4)))
+        return EP_ERR_INVALID_ARG;
+    if (seg == nullptr || rank_off == nullptr || !is_aligned(seg, 4) || !is_aligned(rank_off, 4))
+        return EP_ERR_INVALID_ARG;
+    if (n_rows > 0 && (src_idx == nullptr || !is_aligned(src_idx, 4))) return EP_ERR_INVALID_ARG;
+    if ((out_cnt && !is_aligned(out_cnt, 4)) || (out_rank_tok && !is_aligned(out_rank_tok, 4)) ||
+        (error_word && !is_aligned(error_word, 4)))
+        return EP_ERR_INVALID_ARG;
+
+    // Same tile geometry as ep_layout.
+    int tile_tokens = 128;
+    if ((T + tile_tokens - 1) / tile_tokens > 512)
+        tile_tokens = ((T + 511) / 512 + 31) / 32 * 32;
+    const int ntiles = (T + tile_tokens - 1) / tile_tokens;
+
+    // Scratch words: tile_cnt, tile_rank, per-expert counts, error word.
+    const size_t w_tcnt = (size_t)ntiles * E;
+    const size_t w_trank = (size_t)ntiles * R;
+    const size_t w_cnt = (size_t)E;
+    const size_t need = w_tcnt + w_trank + w_cnt + 1;
+    if (need > (size_t)EP_NOALLOC_SCRATCH_WORDS) return EP_ERR_SCRATCH_LIMIT;
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return status_of(e);
+    DeviceInfo info;
+    if ((e = device_info(dev, &info)) != cudaSuccess) return status_of(e);
+    if (info.cc_major != 10) return EP_ERR_NO_DEVICE;
+    int32_t *scratch = nullptr;
+    const ep_status st = scratch_for_device(dev, &scratch);
+    if (st != EP_OK) return st;
+
+    LayoutArgs a{};
+    a.topk_idx = topk_idx;
+    a.T = T; a.k = k; a.E = E; a.R = R; a.epr = E / R; a.align = A; a.capacity = C;
+    a.tile_tokens = tile_tokens;
+    a.ntiles = ntiles;
+    a.sub_tokens = std::max(1, std::min(tile_tokens, 4096 / R));
+    a.scan_parts_e = std::max(1, std::min(std::max(ntiles, 1), 1024 / E));
+    a.scan_parts_r = std::max(1, std::min(std::max(ntiles, 1), 1024 / R));
+    a.pos_warps = std::min(8, std::max(1, 12288 / E));
+    a.n_rows = (int64_t)n_rows;
+    a.pos = pos;
+    a.src_idx = src_idx;
+    a.seg = seg;
+    a.rank_off = rank_off;
+    a.tile_cnt = scratch;
+    a.tile_rank = scratch + w_tcnt;
+    a.cnt = scratch + w_tcnt + w_trank;
+    a.err = error_word != nullptr ? error_word
+                                  : reinterpret_cast<uint32_t *>(scratch + w_tcnt + w_trank + w_cnt);
+    a.out_cnt = out_cnt;
+    a.out_rank_tok = out_rank_tok;
+    a.out_in_rank = out_in_rank;
+
+    e = cudaMemsetAsync(a.err, 0, 4, stream);
+    if (e == cudaSuccess) e = launch_layout(a, stream);
+    return status_of(e);
+}

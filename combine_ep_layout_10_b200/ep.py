@@ -28,12 +28,13 @@ EP_ERR_CUDA = 4
 EP_ERR_OOM = 5
 EP_ERR_TIMEOUT = 6
 EP_ERR_NO_DEVICE = 7
+EP_ERR_SCRATCH_LIMIT = 8
 
 #: Every symbol the ABI exports (include/ep.h).
 ABI_SYMBOLS = (
     "ep_status_str", "ep_max_recv_rows", "ep_layout", "ep_dispatch", "ep_combine",
     "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
-    "ep_handle_check",
+    "ep_handle_check", "ep_layout_noalloc",
 )
 
 
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.ep_handle_counts_host.restype = I
         L.ep_handle_check.argtypes = [P, P]
         L.ep_handle_check.restype = I
+        L.ep_layout_noalloc.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
+        L.ep_layout_noalloc.restype = I
         _LIB = L
     return _LIB
 
@@ -250,3 +253,28 @@ def ep_combine(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,
 
 def ep_handle_free(handle: Handle) -> None:
     handle.free()
+
+
+def ep_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_ranks: int,
+                      pos: torch.Tensor, src_idx: torch.Tensor, seg: torch.Tensor,
+                      rank_off: torch.Tensor, expert_alignment: int = 1, capacity: int = 0, *,
+                      num_tokens_per_expert: Optional[torch.Tensor] = None,
+                      num_tokens_per_rank: Optional[torch.Tensor] = None,
+                      is_token_in_rank: Optional[torch.Tensor] = None,
+                      error_word: Optional[torch.Tensor] = None, stream=None) -> None:
+    """The layout into caller-owned buffers only (see ep_layout_noalloc in
+    include/ep.h): for callers that cannot allocate device memory.  This
+    wrapper allocates nothing either; every buffer is passed in."""
+    T, k = topk_idx.shape
+    rows = ep_max_recv_rows(T, k, num_experts, expert_alignment, capacity)
+    st = lib().ep_layout_noalloc(
+        _dev_ptr(topk_idx, torch.int32, "topk_idx"), T, k, num_experts, num_ranks,
+        expert_alignment, capacity,
+        _dev_ptr(num_tokens_per_expert, torch.int32, "num_tokens_per_expert", (num_experts,)),
+        _dev_ptr(num_tokens_per_rank, torch.int32, "num_tokens_per_rank", (num_ranks,)),
+        _dev_ptr(is_token_in_rank, torch.uint8, "is_token_in_rank", (T, num_ranks)),
+        _dev_ptr(pos, torch.int32, "pos", (T, k)), _dev_ptr(src_idx, torch.int32, "src_idx", (rows,)),
+        _dev_ptr(seg, torch.int32, "seg", (num_experts + 1,)),
+        _dev_ptr(rank_off, torch.int32, "rank_off", (num_ranks + 1,)),
+        _dev_ptr(error_word, torch.int32, "error_word", (1,)), _stream(stream))
+    _check(st, "ep_layout_noalloc")

@@ -79,7 +79,8 @@ typedef enum ep_status {
     EP_ERR_CUDA = 4,          /* a CUDA runtime call failed */
     EP_ERR_OOM = 5,           /* device allocation failed */
     EP_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up */
-    EP_ERR_NO_DEVICE = 7      /* no CUDA device, or the device is not sm_100 */
+    EP_ERR_NO_DEVICE = 7,     /* no CUDA device, or the device is not sm_100 */
+    EP_ERR_SCRATCH_LIMIT = 8  /* ep_layout_noalloc: the problem needs more than its fixed scratch */
 } ep_status;
 
 /* Human-readable name of a status.  Never NULL; static storage. */
@@ -173,6 +174,48 @@ ep_status ep_handle_counts_host(const ep_handle *handle, int32_t *host_counts,
  * so far.  Synchronises `stream`.  Returns EP_OK, EP_ERR_BAD_EXPERT_ID,
  * EP_ERR_CAPACITY or EP_ERR_TIMEOUT (the first set, in that order). */
 ep_status ep_handle_check(const ep_handle *handle, ep_stream_t stream);
+
+/* Size, in 32-bit words, of the fixed device scratch array ep_layout_noalloc
+ * uses (1 MiB).  Every GPU that loads the library holds it until the process
+ * exits. */
+#define EP_NOALLOC_SCRATCH_WORDS (1 << 18)
+
+/* ep_layout_noalloc -- the routing layout of ep_layout, for callers that
+ * cannot allocate device memory.  The pages have no counterpart: DeepEP's
+ * buffer object allocates its own memory; this entry point exists for users
+ * of this library whose device memory is planned up front (a static memory
+ * planner in a serving loop), who run under another framework's allocator and
+ * may not call the CUDA allocator themselves, or who cannot afford
+ * cudaMalloc's implicit synchronisation on a latency-critical path.
+ *
+ * It computes exactly what ep_layout computes, bit for bit, but returns no
+ * handle: the metadata a handle would own goes to caller buffers instead.
+ *   pos:      device int32 [T, k]          (receive row of each slot, -1 if unused)
+ *   src_idx:  device int32 [rows]          (rows = ep_max_recv_rows(...); -1 on padding)
+ *   seg:      device int32 [E+1];  rank_off: device int32 [R+1]
+ *   num_tokens_per_expert, num_tokens_per_rank, is_token_in_rank: as in
+ *     ep_layout, each may be NULL.
+ *   error_word: device uint32 [1] or NULL.  Cleared by the call, then set
+ *     like a handle's error word (bit 1: id outside [-1, E); bit 2: padded
+ *     expert over capacity).  With NULL, device-detected data errors are not
+ *     reported.
+ * Allocates nothing: no cudaMalloc / cudaMallocAsync / cudaFree and no
+ * allocating library routine.  Its only device memory besides the caller's
+ * buffers is a fixed scratch array of EP_NOALLOC_SCRATCH_WORDS words inside
+ * the library; a problem whose per-tile count matrices need more
+ * (about ceil(T/128) * (E + R) + E + 1 words) is rejected with
+ * EP_ERR_SCRATCH_LIMIT before anything is enqueued.  The first call on a
+ * device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture.  All calls
+ * share the array and it keeps the last call's contents: calls whose GPU work
+ * overlaps (unordered streams) race on it; calls ordered on one stream do not.
+ * Other limits and argument errors as for ep_layout. */
+ep_status ep_layout_noalloc(const int32_t *topk_idx, int num_tokens, int num_topk,
+                            int num_experts, int num_ranks, int expert_alignment, int capacity,
+                            int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                            uint8_t *is_token_in_rank, int32_t *pos, int32_t *src_idx,
+                            int32_t *seg, int32_t *rank_off, uint32_t *error_word,
+                            ep_stream_t stream);
 
 #ifdef __cplusplus
 }
