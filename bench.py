@@ -2,9 +2,9 @@
 """Benchmark of the MoE layout -> dispatch -> combine hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--no-cpu-baseline] [--no-e2e]
+                    [--impl ours|reference] [--no-cpu-baseline] [--no-e2e] [--no-decode]
 
-A step is one pass of the whole path over one batch: ep_layout (3 kernels),
+A step is one pass of the whole path over one batch: ep_layout (2 kernels),
 ep_dispatch (FP8 e4m3 or BF16), ep_combine (BF16), all through the C ABI.
 The default workload is the one the metric is quoted on: 8192 tokens,
 hidden 7168, top-8 of 256 experts with group-limited gating (8 groups, top-4
@@ -42,22 +42,29 @@ sys.path.insert(0, ROOT)
 from combine_ep_layout_10_b200 import workloads as W  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
+GPU_LEAD_CYCLES = 1_000_000  # ~0.5 ms spin before each timed step
+LAUNCHES_PER_STEP = 4        # layout: count, pos; dispatch; combine
 HBM_FALLBACK_GBS = 6650.0
 
 # DRAM traffic per launch from one ncu capture, keyed by the sha256 of the
 # kernel source it was taken on (stale -> reported as null).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # one "ncu --set full" capture of one launch each on the metric workload
+    ("group_limited", "combine"): {"sha": "bf4a5eb031b55673", "bytes": 940059648 + 73684224},
+    ("group_limited", "dispatch"): {"sha": "8dcb1a902f506325", "bytes": 117851648 + 426448384},
+}
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default=W.METRIC_WORKLOAD, choices=sorted(W.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
 
@@ -99,59 +106,83 @@ def source_sha(name: str) -> str:
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    """SM clock and clock-event reasons sampled every 10 ms by NVML (reads
+    only) on the benchmark's GPU; nvidia-smi at 100 ms if NVML is missing."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device_index: int):
         self.dev = device_index
-        self.proc = None
-        self.lines = []
+        self.samples = []          # (wall time, sm MHz, max sm MHz, reasons bitmask)
+        self._stop = threading.Event()
         self.thread = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.dev)
+        bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            nv, h = self._nvml_handle()
+            reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.source = "nvml"
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                             smax, int(reasons_fn(h))))
+                    except Exception:
+                        pass
+                    time.sleep(0.01)
         except Exception:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi"
+            fields = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+                      "clocks_event_reasons.hw_thermal_slowdown",
+                      "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+            def run():
+                try:
+                    proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev),
+                                             "--query-gpu=" + ",".join(fields),
+                                             "--format=csv,noheader,nounits", "-lms", "100"],
+                                            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                except Exception:
+                    return
+                bits = [0x8, 0x40, 0x20, 0x4]
+                for line in proc.stdout:
+                    parts = [q.strip() for q in line.split(",")]
+                    try:
+                        mask = sum(b for b, v in zip(bits, parts[2:]) if v.lower().startswith("active"))
+                        self.samples.append((time.time(), float(parts[0]), float(parts[1]), mask))
+                    except (ValueError, IndexError):
+                        pass
+                    if self._stop.is_set():
+                        break
+                proc.terminate()
+        self.thread = threading.Thread(target=run, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+    def stop(self, window=None) -> dict:
+        """Summarise the samples taken inside `window` (wall-clock start, end)."""
+        self._stop.set()
         if self.thread:
-            self.thread.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:]):
-                if val.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            self.thread.join(timeout=5)
+        sel = [x for x in self.samples if window is None or window[0] <= x[0] <= window[1]]
+        reasons = sorted(n for n, b in self.REASONS.items() if any(x[3] & b for x in sel))
+        return {"sm_mhz": statistics.median(x[1] for x in sel) if sel else None,
+                "sm_max_mhz": max(x[2] for x in sel) if sel else None,
+                "reasons": reasons, "samples": len(sel), "source": self.source}
 
 
 # ---------------------------------------------------------------------------
@@ -180,22 +211,36 @@ def barrier(world: int):
         dist.barrier()
 
 
-def reduce_max(v: float, world: int) -> float:
+def _reduce(v: float, world: int, op: str) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def reduce_max(v: float, world: int) -> float:
+    """Max over ranks (device times: the slowest replica sets the job time)."""
+    return _reduce(v, world, "max")
 
 
 def reduce_sum(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    """Sum over ranks (bytes: every replica's work counts)."""
+    return _reduce(v, world, "sum")
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each replica draws its own batch."""
+    return base + rank
+
+
+def job_throughput(step_ms_local: float, bytes_per_step_local: float, steps: int, world: int):
+    """Whole-job GB/s: all ranks' algorithmic bytes over the slowest rank's time."""
+    step_ms = reduce_max(step_ms_local, world)
+    total = reduce_sum(bytes_per_step_local * steps, world)
+    return total / (step_ms * steps / 1e3) / 1e9, step_ms
 
 
 # ---------------------------------------------------------------------------
@@ -296,7 +341,8 @@ def workload_config(w: W.Workload, world: int) -> dict:
     return {"workload": w.name, "tokens": w.T, "hidden": w.H, "topk": w.k, "experts": w.E,
             "virtual_ranks": w.R, "dispatch": "fp8_e4m3 (fp32 scale / 128 ch)" if w.fp8 else "bf16",
             "combine": "bf16 (fp32 fma chain)", "capacity": w.capacity, "expert_alignment": w.align,
-            "routing": w.routing, "l2": "flushed before every timed step (256 MiB write)",
+            "routing": w.routing,
+            "l2": "flushed before every timed step (256 MiB write, then 256 MiB read to drain dirty lines)",
             "replicas": world, "parallelism": "replicas (no collective)"}
 
 
@@ -313,7 +359,7 @@ def run_ours(args, w):
         B.build()
     ep.lib()
     dev = torch.device("cuda", local)
-    seed = args.seed + rank
+    seed = replica_seed(args.seed, rank)
     x_cpu, idx_cpu, tw_cpu = W.make_routing(w, seed)
     T, H, k, E, R = w.T, w.H, w.k, w.E, w.R
     n_rows = ep.ep_max_recv_rows(T, k, E, w.align, w.capacity)
@@ -332,67 +378,113 @@ def run_ours(args, w):
     cnt = torch.empty(E, dtype=torch.int32, device=dev)
     rtok = torch.empty(R, dtype=torch.int32, device=dev)
     in_rank = torch.empty(T, R, dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    def flush_l2():
+        # Write a buffer larger than L2, then read another one: the read
+        # evicts the dirty lines (written back here, outside the timed window)
+        # and leaves L2 holding clean, unrelated data.
+        flush_w.zero_()
+        flush_r.sum(dtype=torch.int64)
+
     def step(ev=None):
+        """One layout -> dispatch -> combine.  ev: None, 2 events (step
+        boundaries) or 4 events (one window per call)."""
         if ev is not None:
+            # Let the host run ahead: the step's launches are all queued before
+            # the GPU reaches ev[0], so the windows hold GPU time only (the
+            # host issue time is reported separately as host_us_per_step).
+            torch.cuda._sleep(GPU_LEAD_CYCLES)
             ev[0].record(stream)
         res = ep.ep_layout(idx, E, R, w.align, w.capacity, num_tokens_per_expert=cnt,
                            num_tokens_per_rank=rtok, is_token_in_rank=in_rank)
-        if ev is not None:
+        if ev is not None and len(ev) == 4:
             ev[1].record(stream)
         ep.ep_dispatch(res.handle, x, w.fp8, recv, scales)
-        if ev is not None:
+        if ev is not None and len(ev) == 4:
             ev[2].record(stream)
         ep.ep_combine(res.handle, y, tw, out)
         if ev is not None:
-            ev[3].record(stream)
+            ev[-1].record(stream)
         return res.handle
 
     for _ in range(max(args.warmup, 0)):
-        flush.zero_()
+        flush_l2()
         step().free()
     torch.cuda.synchronize()
     assert step().check() == ep.EP_OK
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Timed region: events at step boundaries only, so that nothing sits between
+    # the step's kernels in the stream (the kernels use programmatic dependent
+    # launch and may overlap their launch with the previous kernel's tail).
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.1)
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    handles = []
+    t0_wall = time.time()
+    last = None
     for i in range(args.steps):
-        flush.zero_()
-        handles.append(step(events[i]))
-        if len(handles) > 4:
-            handles.pop(0).free()
+        flush_l2()
+        h = step(events[i])
+        if last is not None:
+            last.free()
+        last = h
     torch.cuda.synchronize()
     barrier(world)
-    wall = time.perf_counter() - wall0
-    clocks = sampler.stop()
-    status = handles[-1].check()
-    for h in handles:
-        h.free()
+    wall1 = time.perf_counter()
+    wall = wall1 - wall0
+    clocks = sampler.stop(window=(t0_wall, time.time()))
+    status = last.check()
+    last.free()
     if status != ep.EP_OK:
         raise SystemExit("device error: %s" % ep.status_str(status))
 
-    lay = [e[0].elapsed_time(e[1]) for e in events]
-    dis = [e[1].elapsed_time(e[2]) for e in events]
-    com = [e[2].elapsed_time(e[3]) for e in events]
-    stp = [e[0].elapsed_time(e[3]) for e in events]
+    # Host cost of issuing one step through the binding, measured with the GPU
+    # kept busy (no launch-queue back-pressure): the time a caller's CPU spends.
+    host = []
+    for _ in range(10):
+        torch.cuda._sleep(20 * GPU_LEAD_CYCLES)
+        t_issue = time.perf_counter()
+        h = step()
+        host.append(time.perf_counter() - t_issue)
+        torch.cuda.synchronize()
+        h.free()
+    host_s = statistics.median(host)
+
+    stp = [e[0].elapsed_time(e[1]) for e in events]
+
+    # Attribution pass: the same K steps with a window around each call, for
+    # the per-kernel times and the roofline (events between the calls keep the
+    # kernels from overlapping, so these windows add up to a bit more than
+    # the timed step).
+    attr = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    last = None
+    for i in range(args.steps):
+        flush_l2()
+        h = step(attr[i])
+        if last is not None:
+            last.free()
+        last = h
+    torch.cuda.synchronize()
+    last.free()
+    lay = [e[0].elapsed_time(e[1]) for e in attr]
+    dis = [e[1].elapsed_time(e[2]) for e in attr]
+    com = [e[2].elapsed_time(e[3]) for e in attr]
     mean = lambda v: sum(v) / len(v)  # noqa: E731
-    step_ms = reduce_max(mean(stp), world)
+    value, step_ms = job_throughput(mean(stp), nbytes["step"], args.steps, world)
     lay_ms, dis_ms, com_ms = (reduce_max(mean(v), world) for v in (lay, dis, com))
-    total_bytes = reduce_sum(nbytes["step"] * args.steps, world)
-    value = total_bytes / (step_ms * args.steps / 1e3) / 1e9
 
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"]
     kern = {
-        "layout": {"us": lay_ms * 1e3, "bytes": nbytes["layout"], "launches_per_step": 3},
+        "note": "per-call windows from an attribution pass of the same steps",
+        "layout": {"us": lay_ms * 1e3, "bytes": nbytes["layout"], "launches_per_step": 2},
         "dispatch": {"us": dis_ms * 1e3, "bytes": nbytes["dispatch"],
                      "gbs": nbytes["dispatch"] / (dis_ms / 1e3) / 1e9},
         "combine": {"us": com_ms * 1e3, "bytes": nbytes["combine"],
@@ -413,6 +505,10 @@ def run_ours(args, w):
     if not args.no_e2e:
         e2e = run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y, nbytes, world)
 
+    decode = None
+    if not args.no_decode:
+        decode = run_decode_latency(dev, ep)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed)
@@ -425,13 +521,94 @@ def run_ours(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 5 * args.steps, "clocks": clocks, "wall_s": wall,
+            "decode": decode,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "wall_s": wall,
+            "host_us_per_step": host_s * 1e6,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def run_decode_latency(dev, ep, steps: int = 100) -> dict:
+    """Decoding with a cached handle: one layout, then `steps` dispatch +
+    combine calls with new x every step (x for step s drawn from seed
+    1000 + s, staged in device memory beforehand, as a previous layer would
+    leave it).  Reports us per call with plain launches and us per step for
+    a replayed CUDA graph of dispatch + combine."""
+    w = W.WORKLOADS["decode"]
+    _, idx, tw = W.make_routing(w)
+    res = ep.ep_layout(idx.to(dev), w.E, w.R, w.align, w.capacity)
+    h = res.handle
+    rows = h.num_recv_rows
+    xs = torch.stack([W.make_x(w, 1000 + s) for s in range(steps)]).to(dev)
+    xb = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    recv = torch.empty(rows, w.H, dtype=torch.float8_e4m3fn, device=dev)
+    sc = torch.empty(rows, w.H // 128, dtype=torch.float32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(21)
+    y = torch.randn(rows, w.H, generator=g, device=dev).to(torch.bfloat16)
+    twd = tw.to(dev)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ep.ep_dispatch(h, xb, True, recv, sc)
+        ep.ep_combine(h, y, twd, out)
+
+    for s in range(3):
+        xb.copy_(xs[s])
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for s in range(steps):
+        xb.copy_(xs[s])
+        torch.cuda._sleep(GPU_LEAD_CYCLES // 4)
+        ev[s][0].record(stream)
+        ep.ep_dispatch(h, xb, True, recv, sc)
+        ev[s][1].record(stream)
+        ep.ep_combine(h, y, twd, out)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    d_us = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) * 1e3
+    c_us = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) * 1e3
+
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        step()
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        step()
+    for s in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    total = 0.0
+    for s in range(steps):
+        xb.copy_(xs[s])
+        torch.cuda._sleep(GPU_LEAD_CYCLES // 4)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    status = h.check()
+    del graph
+    h.free()
+    if status != ep.EP_OK:
+        raise SystemExit("decode: device error %s" % ep.status_str(status))
+    V = w.T * w.k
+    disp_bytes = w.T * w.H * 2 + w.T * w.k * 4 + V * w.H + V * (w.H // 128) * 4
+    comb_bytes = V * w.H * 2 + w.T * w.k * 8 + w.T * w.H * 2
+    return {"workload": "decode", "tokens": w.T, "hidden": w.H, "topk": w.k, "experts": w.E,
+            "capacity": w.capacity, "steps": steps, "dispatch_us": d_us, "combine_us": c_us,
+            "step_us_plain": d_us + c_us, "step_us_graph": total / steps * 1e3,
+            "dispatch_bytes": disp_bytes, "combine_bytes": comb_bytes}
 
 
 def run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y_dev, nbytes, world):

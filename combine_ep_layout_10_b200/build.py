@@ -50,12 +50,15 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile and link libep_b200.so if missing or stale; return its path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          out: str | None = None) -> str:
+    """Compile and link libep_b200.so (or `out`, e.g. a variant built with
+    extra -D flags) if missing or stale; return its path."""
+    target = out or LIB
+    if not force and out is None and not _stale():
         return LIB
-    os.makedirs(LIBDIR, exist_ok=True)
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    os.makedirs(os.path.dirname(target), exist_ok=True)
+    tmp = target + ".tmp.%d" % os.getpid()
     cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC, "-shared",
            *sources(), "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -63,8 +66,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("CUDA library build failed:\n%s\n%s%s" % (" ".join(cmd), res.stdout, res.stderr))
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

@@ -22,15 +22,31 @@
 namespace ep {
 namespace {
 
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = EP_COMBINE_THREADS;
 constexpr int kLoadBatch = 8;  // row loads issued back to back before accumulating
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     uint4 r;
+#if EP_COMBINE_L2_PREFETCH
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+#else
     asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
         : "l"(p));
+#endif
     return r;
+}
+
+__device__ __forceinline__ void st_out_v4(void *p, const uint4 &v) {
+#if EP_COMBINE_STREAM_STORE
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+#else
+    *reinterpret_cast<uint4 *>(p) = v;
+#endif
 }
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4 &v) {
@@ -54,6 +70,7 @@ template <int VPT>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
     __shared__ int32_t p_s[kMaxTopk];
     __shared__ float w_s[kMaxTopk];
+    pdl_wait_then_trigger();
     const int t = blockIdx.x / a.blocks_per_token;
     const int cb = blockIdx.x - t * a.blocks_per_token;
     if (threadIdx.x < a.k) {
@@ -88,7 +105,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
         o.y = pack_bf16x2(acc[2], acc[3]);
         o.z = pack_bf16x2(acc[4], acc[5]);
         o.w = pack_bf16x2(acc[6], acc[7]);
-        *reinterpret_cast<uint4 *>(a.out + (size_t)t * row_bytes + (size_t)v * 16) = o;
+        st_out_v4(a.out + (size_t)t * row_bytes + (size_t)v * 16, o);
     }
 }
 
@@ -100,12 +117,11 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
     if ((long long)a.blocks_per_token * a.vpt * kCombineThreads < a.nvec)
         return cudaErrorInvalidConfiguration;
     switch (a.vpt) {
-        case 1: combine_kernel<1><<<(unsigned)blocks, kCombineThreads, 0, s>>>(a); break;
-        case 2: combine_kernel<2><<<(unsigned)blocks, kCombineThreads, 0, s>>>(a); break;
-        case 4: combine_kernel<4><<<(unsigned)blocks, kCombineThreads, 0, s>>>(a); break;
+        case 1: return launch_kernel(combine_kernel<1>, (unsigned)blocks, kCombineThreads, 0, s, a);
+        case 2: return launch_kernel(combine_kernel<2>, (unsigned)blocks, kCombineThreads, 0, s, a);
+        case 4: return launch_kernel(combine_kernel<4>, (unsigned)blocks, kCombineThreads, 0, s, a);
         default: return cudaErrorInvalidConfiguration;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace ep

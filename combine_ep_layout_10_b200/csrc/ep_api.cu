@@ -17,10 +17,36 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 DeviceInfo g_info[kMaxDevices];
 bool g_have[kMaxDevices];
+cudaMemPool_t g_pool[kMaxDevices];
 
-constexpr int kDefaultTileTokens = 128;
-constexpr int kMaxTiles = 512;
-constexpr int kMaxChunkChannels = 8192;
+// Stream-ordered pool for handle metadata, one per device, created on first
+// use and kept for the life of the process.  Its release threshold is
+// unbounded, so memory freed by ep_handle_free stays in the pool and the next
+// layout's allocation is pure bookkeeping (the default pool would return it
+// to the driver at every synchronisation and map it again).
+cudaError_t handle_pool(int device, cudaMemPool_t *out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_pool[device] == nullptr) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = device;
+        cudaMemPool_t pool = nullptr;
+        cudaError_t e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~0ull;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return e;
+        }
+        g_pool[device] = pool;
+    }
+    *out = g_pool[device];
+    return cudaSuccess;
+}
+
+constexpr int kMaxChunkChannels = EP_DISPATCH_MAX_CHUNK;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -114,10 +140,8 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     ep_status st = current_device(&dev, &info);
     if (st != EP_OK) return st;
 
-    int tile_tokens = kDefaultTileTokens;
-    if ((T + tile_tokens - 1) / tile_tokens > kMaxTiles)
-        tile_tokens = (int)round_up((size_t)((T + kMaxTiles - 1) / kMaxTiles), 32);
-    const int ntiles = (T + tile_tokens - 1) / tile_tokens;
+    const LayoutGeometry geo = layout_geometry(T, k, E, R);
+    const int ntiles = geo.ntiles;
 
     // One stream-ordered allocation, every array 256-byte aligned.
     size_t off = 0;
@@ -134,8 +158,11 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     const size_t o_cnt = carve((size_t)E * 4);
     const size_t o_tcnt = carve((size_t)ntiles * E * 4);
     const size_t o_trank = carve((size_t)ntiles * R * 4);
+    const size_t o_terr = carve((size_t)ntiles * 4);
     void *block = nullptr;
-    cudaError_t e = cudaMallocAsync(&block, off, stream);
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = handle_pool(dev, &pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&block, off, pool, stream);
     if (e != cudaSuccess) return cuda_status(e);
 
     ep_handle *h = new (std::nothrow) ep_handle;
@@ -146,7 +173,7 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     unsigned char *b = static_cast<unsigned char *>(block);
     h->T = T; h->k = k; h->E = E; h->R = R; h->align = A; h->capacity = C;
     h->experts_per_rank = E / R;
-    h->tile_tokens = tile_tokens;
+    h->tile_tokens = geo.tile_tokens;
     h->ntiles = ntiles;
     h->n_rows = (int64_t)n_rows;
     h->device = dev;
@@ -160,25 +187,25 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     h->cnt = reinterpret_cast<int32_t *>(b + o_cnt);
     h->tile_cnt = reinterpret_cast<int32_t *>(b + o_tcnt);
     h->tile_rank = reinterpret_cast<int32_t *>(b + o_trank);
+    h->tile_err = reinterpret_cast<uint32_t *>(b + o_terr);
 
     LayoutArgs a{};
     a.topk_idx = topk_idx;
     a.T = T; a.k = k; a.E = E; a.R = R; a.epr = E / R; a.align = A; a.capacity = C;
-    a.tile_tokens = tile_tokens;
+    a.tile_tokens = geo.tile_tokens;
     a.ntiles = ntiles;
-    a.sub_tokens = std::max(1, std::min(tile_tokens, 4096 / R));
-    a.scan_parts_e = std::max(1, std::min(std::max(ntiles, 1), 1024 / E));
-    a.scan_parts_r = std::max(1, std::min(std::max(ntiles, 1), 1024 / R));
-    a.pos_warps = std::min(8, std::max(1, 12288 / E));
+    a.sub_tokens = geo.sub_tokens;
+    a.pos_warps = geo.pos_warps;
+    a.ids_in_smem = geo.ids_in_smem;
     a.n_rows = (int64_t)n_rows;
     a.pos = h->pos; a.src_idx = h->src_idx; a.seg = h->seg; a.rank_off = h->rank_off;
-    a.cnt = h->cnt; a.tile_cnt = h->tile_cnt; a.tile_rank = h->tile_rank; a.err = h->err;
+    a.cnt = h->cnt; a.tile_cnt = h->tile_cnt; a.tile_rank = h->tile_rank;
+    a.tile_err = h->tile_err; a.err = h->err;
     a.out_cnt = out_cnt;
     a.out_rank_tok = out_rank_tok;
     a.out_in_rank = out_in_rank;
 
-    e = cudaMemsetAsync(h->err, 0, 4, stream);
-    if (e == cudaSuccess) e = launch_layout(a, stream);
+    e = launch_layout(a, stream);  // also (re)initialises the error word
     if (e != cudaSuccess) {
         cudaFreeAsync(block, stream);
         delete h;
@@ -215,13 +242,11 @@ ep_status ep_dispatch(const ep_handle *h, const void *x, int H, int use_fp8, voi
     a.pos = h->pos;
     a.recv = static_cast<uint8_t *>(recv_x);
     a.scales = recv_scales;
-    a.err = h->err;
     a.T = h->T; a.k = h->k; a.H = H;
     a.chunk = chunk;
     a.nchunks = (H + chunk - 1) / chunk;
     a.nunits = (long long)h->T * a.nchunks;
-    a.stages = use_fp8 ? 3 : 4;
-    cudaError_t e = launch_dispatch(a, use_fp8 != 0, info.num_sms, stream);
+    cudaError_t e = launch_dispatch(a, use_fp8 != 0, stream);
     if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)
         e = cudaMemcpyAsync(recv_src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
     return cuda_status(e);
@@ -248,8 +273,8 @@ ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int
     a.out = static_cast<uint8_t *>(out);
     a.T = h->T; a.k = h->k; a.H = H;
     a.nvec = H / 8;
-    a.vpt = 1;
-    a.blocks_per_token = (a.nvec + 127) / 128;
+    a.vpt = EP_COMBINE_VPT;
+    a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
     return cuda_status(launch_combine(a, stream));
 }
 

@@ -9,18 +9,68 @@
 
 #include "ep.h"
 
+// Launch-shape parameters, chosen by measurement on B200.  Each can be
+// overridden with -D at build time to sweep it.
+#ifndef EP_DISPATCH_MAX_CHUNK     // dispatch: at most this many channels per work unit
+#define EP_DISPATCH_MAX_CHUNK 8192
+#endif
+#ifndef EP_COMBINE_THREADS        // threads per combine block
+#define EP_COMBINE_THREADS 128
+#endif
+#ifndef EP_COMBINE_VPT            // combine: 16-byte vectors per thread (1, 2 or 4)
+#define EP_COMBINE_VPT 1
+#endif
+#ifndef EP_COMBINE_L2_PREFETCH    // combine: add the .L2::256B prefetch hint to the row loads
+#define EP_COMBINE_L2_PREFETCH 0
+#endif
+#ifndef EP_COMBINE_STREAM_STORE   // combine: evict-first (.cs) stores of the output
+#define EP_COMBINE_STREAM_STORE 0
+#endif
+
+#ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
+#define EP_USE_PDL 1
+#endif
+
 namespace ep {
+
+// Programmatic dependent launch (sm_90+).  Every kernel of the library is
+// launched with programmatic stream serialisation, so the GPU may schedule it
+// while the previous kernel in the stream is still finishing; the first thing
+// each kernel does is pdl_wait(), which returns once the previous grid has
+// completed and its memory is visible, so no input is read early.  It then
+// lets its own dependents be scheduled.  The saving is the launch latency
+// between back-to-back kernels.
+__device__ __forceinline__ void pdl_wait_then_trigger() {
+#if EP_USE_PDL
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = EP_USE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Bits of the handle's device error word.
 constexpr uint32_t kErrBadExpertId = 1u;
 constexpr uint32_t kErrCapacity = 2u;
-constexpr uint32_t kErrTimeout = 4u;
+constexpr uint32_t kErrTimeout = 4u;  // reserved: no kernel waits on another today
 
 constexpr int kMaxTopk = 32;
 constexpr int kMaxExperts = 4096;
 
-// Bounded device waits give up after about a second at B200 clocks.
-constexpr long long kWaitLimitCycles = 2000000000LL;
 
 }  // namespace ep
 
@@ -38,21 +88,55 @@ struct ep_handle {
     int32_t *seg;            // [E+1]
     int32_t *rank_off;       // [R+1]
     int32_t *cnt;            // [E]
-    int32_t *tile_cnt;       // [ntiles*E]  per-tile expert counts, then exclusive bases
-    int32_t *tile_rank;      // [ntiles*R]  per-tile token-in-rank counts
+    int32_t *tile_cnt;       // [ntiles*E]  per-tile expert counts (scratch)
+    int32_t *tile_rank;      // [ntiles*R]  per-tile token-in-rank counts (scratch)
+    uint32_t *tile_err;      // [ntiles]    per-tile bad-id flags (scratch)
     uint32_t *err;           // [1] device error word
 };
 
 namespace ep {
 
+__host__ __device__ constexpr int align4(int n) { return (n + 3) & ~3; }
+
+// Tile geometry of the layout.  Tiles of 128 tokens (doubled until the
+// [tiles x (E + R)] count matrices fit the position kernel's shared memory);
+// count-kernel rank-bitmask sub-blocks of at most 12288 words; position-kernel
+// warps whose per-warp count rows fit 12288 words; the tile's ids staged in
+// shared memory when they fit.
+constexpr int kLayoutMatWords = 24576;
+struct LayoutGeometry {
+    int tile_tokens, ntiles, sub_tokens, pos_warps;
+    bool ids_in_smem;  // the position kernel stages the tile's ids in shared memory
+};
+// Shared-memory words of the position kernel.
+inline int layout_pos_smem_words(int ntiles, int E, int R, int pos_warps, int id_words) {
+    return align4(ntiles * E) + align4(ntiles * R) + 2 * align4(E) + align4(E + 1) +
+           align4(pos_warps * E) + id_words;
+}
+inline LayoutGeometry layout_geometry(int T, int k, int E, int R) {
+    LayoutGeometry g;
+    g.tile_tokens = 128;
+    while ((int64_t)((T + g.tile_tokens - 1) / g.tile_tokens) * (E + R) > kLayoutMatWords &&
+           g.tile_tokens < (1 << 29))
+        g.tile_tokens *= 2;
+    g.ntiles = (T + g.tile_tokens - 1) / g.tile_tokens;
+    const int rw = (R + 31) / 32;
+    g.sub_tokens = 12288 / rw < g.tile_tokens ? 12288 / rw : g.tile_tokens;
+    g.pos_warps = 12288 / E >= 8 ? 8 : (12288 / E > 0 ? 12288 / E : 1);
+    const int64_t id_words = (int64_t)g.tile_tokens * k;
+    g.ids_in_smem = id_words <= 8192 &&
+                    layout_pos_smem_words(g.ntiles, E, R, g.pos_warps, (int)id_words) <= 50000;
+    return g;
+}
+
 struct LayoutArgs {
     const int32_t *topk_idx;
     int T, k, E, R, epr, align, capacity;
-    int tile_tokens, ntiles, sub_tokens;
-    int scan_parts_e, scan_parts_r, pos_warps;
+    int tile_tokens, ntiles, sub_tokens, pos_warps;
+    bool ids_in_smem;
     int64_t n_rows;
     int32_t *pos, *src_idx, *seg, *rank_off, *cnt, *tile_cnt, *tile_rank;
-    uint32_t *err;
+    uint32_t *tile_err, *err;
     int32_t *out_cnt, *out_rank_tok;
     uint8_t *out_in_rank;
 };
@@ -62,12 +146,10 @@ struct DispatchArgs {
     const int32_t *pos;      // [T, k]
     uint8_t *recv;           // [rows, H] bf16 or e4m3
     float *scales;           // [rows, H/128] (FP8 only)
-    uint32_t *err;
     int T, k, H;
-    int chunk;               // channels per work unit
+    int chunk;               // channels per work unit (block)
     int nchunks;             // units per token
     long long nunits;        // T * nchunks
-    int stages;              // input ring depth
 };
 
 struct CombineArgs {
@@ -83,7 +165,9 @@ struct CombineArgs {
 
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
-cudaError_t launch_dispatch(const DispatchArgs &a, bool fp8, int num_sms, cudaStream_t s);
+size_t layout_count_smem(const LayoutArgs &a);
+size_t layout_pos_smem(const LayoutArgs &a);
+cudaError_t launch_dispatch(const DispatchArgs &a, bool fp8, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 
 // Per-device facts, cached.

@@ -6,115 +6,35 @@
 // news.hada.io, "Patrones de uso en entrenamiento, prefill y decoding": the
 // handle carries the routing metadata and the per-expert counts).  Receive
 // rows are expert-major and, inside an expert, in (source token, slot) order,
-// so every position is a pure function of topk_idx: three kernels, no
-// inter-CTA waits and no atomics whose order could leak into a position.
+// so every position is a pure function of topk_idx.  Two kernels, no
+// inter-CTA waits, no atomics whose order could leak into a position:
 //
 //   1. layout_count_kernel (one CTA per tile of tokens): per-tile expert
-//      histogram (shared-memory integer atomics: the result of an integer
-//      sum does not depend on the order), token-in-rank flags and per-tile
-//      rank counts.
-//   2. layout_scan_kernel (one CTA): per-expert exclusive scan over tiles,
-//      expert totals, segment offsets (block-wide scan), rank slices, rank
-//      counts, capacity check, -1 fill of padding rows.
-//   3. layout_pos_kernel (one CTA per tile): within-tile ranks in slot order
-//      with warp __match_any_sync + popc, a prefix over the CTA's warps, and
-//      the tile base from step 2; writes pos[t][j] and src_idx[row].
+//      histogram (shared-memory integer atomics: an integer sum does not
+//      depend on the order), token-in-rank flags, per-tile rank counts and a
+//      per-tile bad-id flag.
+//   2. layout_pos_kernel (one CTA per tile): loads the whole [tiles x E]
+//      count matrix into shared memory, derives its own tile base and the
+//      global segment offsets from it (every CTA does this redundantly: a few
+//      tens of KB from L2 per CTA instead of a serial single-CTA scan kernel),
+//      then ranks its slots in slot order with warp __match_any_sync + popc
+//      and a prefix over its warps, and writes pos[t][j] and src_idx[row].
+//      CTA 0 publishes counts, segments, rank slices, rank counts and the
+//      error word; the -1 fill of padding rows is spread over all CTAs.
 #include "ep_internal.cuh"
 
 namespace ep {
 namespace {
 
 constexpr int kCountThreads = 256;
-constexpr int kScanThreads = 1024;
 constexpr int kPosThreads = 256;
 
-__device__ __forceinline__ int load_id(const LayoutArgs &a, int64_t s, bool report) {
-    int e = __ldg(a.topk_idx + s);
-    if (e < -1 || e >= a.E) {
-        if (report) atomicOr(a.err, kErrBadExpertId);
-        e = -1;
-    }
-    return e;
-}
-
-// ---------------------------------------------------------------------------
-// 1. per-tile counts and token-in-rank flags
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kCountThreads) layout_count_kernel(LayoutArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    int32_t *cnt_s = reinterpret_cast<int32_t *>(smem);           // [E]
-    int32_t *rcnt_s = cnt_s + a.E;                                // [R]
-    uint32_t *flag_s = reinterpret_cast<uint32_t *>(rcnt_s + a.R);  // [sub_tokens * R]
-
-    const int tile = blockIdx.x;
-    const int t0 = tile * a.tile_tokens;
-    const int nt = min(a.tile_tokens, a.T - t0);
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x) cnt_s[i] = 0;
-    for (int i = threadIdx.x; i < a.R; i += blockDim.x) rcnt_s[i] = 0;
-
-    for (int sb = 0; sb < nt; sb += a.sub_tokens) {
-        const int ns = min(a.sub_tokens, nt - sb);
-        const int nflags = ns * a.R;
-        for (int i = threadIdx.x; i < nflags; i += blockDim.x) flag_s[i] = 0u;
-        __syncthreads();
-
-        const int64_t s0 = (int64_t)(t0 + sb) * a.k;
-        const int nslots = ns * a.k;
-        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
-            const int e = load_id(a, s0 + s, true);
-            if (e < 0) continue;
-            atomicAdd(&cnt_s[e], 1);
-            const int r = e / a.epr;
-            // Only the first slot of a token that lands on rank r counts the token.
-            if (atomicExch(&flag_s[(s / a.k) * a.R + r], 1u) == 0u) atomicAdd(&rcnt_s[r], 1);
-        }
-        __syncthreads();
-
-        if (a.out_in_rank != nullptr) {
-            uint8_t *dst = a.out_in_rank + (int64_t)(t0 + sb) * a.R;
-            if ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0 && (nflags & 3) == 0) {
-                uint32_t *dw = reinterpret_cast<uint32_t *>(dst);
-                for (int i = threadIdx.x; i < nflags / 4; i += blockDim.x) {
-                    const uint32_t *f = flag_s + 4 * i;
-                    dw[i] = f[0] | (f[1] << 8) | (f[2] << 16) | (f[3] << 24);
-                }
-            } else {
-                for (int i = threadIdx.x; i < nflags; i += blockDim.x) dst[i] = (uint8_t)flag_s[i];
-            }
-        }
-        __syncthreads();
-    }
-
-    int32_t *tc = a.tile_cnt + (int64_t)tile * a.E;
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x) tc[i] = cnt_s[i];
-    int32_t *tr = a.tile_rank + (int64_t)tile * a.R;
-    for (int i = threadIdx.x; i < a.R; i += blockDim.x) tr[i] = rcnt_s[i];
-}
-
-// ---------------------------------------------------------------------------
-// 2. scans
-// ---------------------------------------------------------------------------
-
-// Column partial sums of mat[ntiles][C] split into P contiguous tile ranges:
-// part[p*C + c] = sum of mat[tile][c] over the p-th range.
-__device__ void column_partials(const int32_t *mat, int ntiles, int C, int P, int32_t *part) {
-    for (int item = threadIdx.x; item < P * C; item += blockDim.x) {
-        const int c = item % C;
-        const int p = item / C;
-        const int lo = (int)((int64_t)p * ntiles / P);
-        const int hi = (int)((int64_t)(p + 1) * ntiles / P);
-        int32_t s = 0;
-#pragma unroll 8
-        for (int t = lo; t < hi; ++t) s += mat[(int64_t)t * C + c];
-        part[p * C + c] = s;
-    }
-}
-
-// Exclusive scan of v over the whole block (blockDim.x == kScanThreads);
-// returns the exclusive prefix of this thread's value and the block total.
+// Exclusive scan of one value per thread over the block (blockDim.x <= 1024);
+// returns the exclusive prefix and writes the block total to *total.
 __device__ int32_t block_exclusive_scan(int32_t v, int32_t *total, int32_t *warp_s) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    const int nwarps = (blockDim.x + 31) >> 5;
     int32_t incl = v;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -124,14 +44,14 @@ __device__ int32_t block_exclusive_scan(int32_t v, int32_t *total, int32_t *warp
     if (lane == 31) warp_s[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int32_t w = warp_s[lane];  // kScanThreads / 32 == 32 warps
+        const int32_t w = (lane < nwarps) ? warp_s[lane] : 0;
         int32_t wi = w;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const int32_t n = __shfl_up_sync(0xffffffffu, wi, d);
             if (lane >= d) wi += n;
         }
-        warp_s[lane] = wi - w;      // exclusive warp offsets
+        warp_s[lane] = wi - w;
         if (lane == 31) warp_s[32] = wi;
     }
     __syncthreads();
@@ -141,45 +61,148 @@ __device__ int32_t block_exclusive_scan(int32_t v, int32_t *total, int32_t *warp
     return excl;
 }
 
-__global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a) {
+// Copy n int32 words global -> shared (16-byte vectors when both are aligned).
+__device__ __forceinline__ void load_words(int32_t *dst, const int32_t *src, int n) {
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+        const int n4 = n >> 2;
+        const int4 *s4 = reinterpret_cast<const int4 *>(src);
+        int4 *d4 = reinterpret_cast<int4 *>(dst);
+        for (int i = threadIdx.x; i < n4; i += blockDim.x) d4[i] = __ldg(s4 + i);
+        for (int i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) dst[i] = __ldg(src + i);
+    } else {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = __ldg(src + i);
+    }
+}
+
+// Id of slot s of the tile (-1 for unused or invalid ids), from shared memory
+// when the tile's ids were staged there.
+__device__ __forceinline__ int tile_id(const LayoutArgs &a, const int32_t *ids_s, int64_t s0, int s) {
+    int e = a.ids_in_smem ? ids_s[s] : __ldg(a.topk_idx + s0 + s);
+    if (e < -1 || e >= a.E) e = -1;
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// 1. per-tile counts and token-in-rank flags
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCountThreads) layout_count_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int E = a.E, R = a.R;
-    const int partE = a.scan_parts_e * E;
-    const int partR = a.scan_parts_r * R;
-    int32_t *part = reinterpret_cast<int32_t *>(smem);        // [max(partE, partR)]
-    int32_t *cnt_s = part + max(partE, partR);                 // [E]
-    int32_t *seg_s = cnt_s + E;                                // [E+1]
+    pdl_wait_then_trigger();
+    const int RW = (a.R + 31) >> 5;                                 // mask words per token
+    int32_t *cnt_s = reinterpret_cast<int32_t *>(smem);             // [E]
+    int32_t *rcnt_s = cnt_s + a.E;                                  // [R]
+    uint32_t *mask_s = reinterpret_cast<uint32_t *>(rcnt_s + a.R);  // [sub_tokens][RW] rank bits
+    int32_t *ids_s = reinterpret_cast<int32_t *>(mask_s) + align4(a.sub_tokens * RW);  // [tile ids]
+
+    const int tile = blockIdx.x;
+    const int t0 = tile * a.tile_tokens;
+    const int nt = min(a.tile_tokens, a.T - t0);
+    const int64_t s_tile = (int64_t)t0 * a.k;
+    if (a.ids_in_smem) load_words(ids_s, a.topk_idx + s_tile, nt * a.k);
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) cnt_s[i] = 0;
+    for (int i = threadIdx.x; i < a.R; i += blockDim.x) rcnt_s[i] = 0;
+    int bad = 0;
+
+    for (int sb = 0; sb < nt; sb += a.sub_tokens) {
+        const int ns = min(a.sub_tokens, nt - sb);
+        for (int i = threadIdx.x; i < ns * RW; i += blockDim.x) mask_s[i] = 0u;
+        __syncthreads();
+
+        const int sub0 = sb * a.k;  // first slot of the sub-block inside the tile
+        const int nslots = ns * a.k;
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            int e = a.ids_in_smem ? ids_s[sub0 + s] : __ldg(a.topk_idx + s_tile + sub0 + s);
+            if (e < -1 || e >= a.E) e = -2;  // invalid id: counted as unused, flagged
+            if (e < 0) {
+                bad |= (e == -2);
+                continue;
+            }
+            atomicAdd(&cnt_s[e], 1);
+            const int r = e / a.epr;
+            const uint32_t bit = 1u << (r & 31);
+            // The slot that sets the token's bit for rank r counts the token.
+            if (!(atomicOr(&mask_s[(s / a.k) * RW + (r >> 5)], bit) & bit)) atomicAdd(&rcnt_s[r], 1);
+        }
+        __syncthreads();
+
+        if (a.out_in_rank != nullptr) {
+            const int nflags = ns * a.R;
+            uint8_t *dst = a.out_in_rank + (int64_t)(t0 + sb) * a.R;
+            if ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0 && (a.R & 3) == 0) {
+                // One warp per token row; lane w writes flags 4w..4w+3 as one word
+                // (a multiple of 4 never straddles a 32-bit mask word).
+                const int words = a.R >> 2;
+                const int lane = threadIdx.x & 31;
+                for (int tl = threadIdx.x >> 5; tl < ns; tl += blockDim.x >> 5) {
+                    uint32_t *dw = reinterpret_cast<uint32_t *>(dst + (int64_t)tl * a.R);
+                    const uint32_t *mrow = mask_s + tl * RW;
+                    for (int w4 = lane; w4 < words; w4 += 32) {
+                        const uint32_t m = mrow[w4 >> 3] >> ((w4 & 7) * 4);
+                        dw[w4] = (m & 1u) | ((m & 2u) << 7) | ((m & 4u) << 14) | ((m & 8u) << 21);
+                    }
+                }
+            } else {
+                for (int i = threadIdx.x; i < nflags; i += blockDim.x) {
+                    const int tl = i / a.R;
+                    const int r = i - tl * a.R;
+                    dst[i] = (uint8_t)((mask_s[tl * RW + (r >> 5)] >> (r & 31)) & 1u);
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    bad = __syncthreads_or(bad);
+    int32_t *tc = a.tile_cnt + (int64_t)tile * a.E;
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) tc[i] = cnt_s[i];
+    int32_t *tr = a.tile_rank + (int64_t)tile * a.R;
+    for (int i = threadIdx.x; i < a.R; i += blockDim.x) tr[i] = rcnt_s[i];
+    if (threadIdx.x == 0) a.tile_err[tile] = bad ? kErrBadExpertId : 0u;
+}
+
+// ---------------------------------------------------------------------------
+// 2. segments and positions
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int E = a.E, R = a.R, W = a.pos_warps, NT = a.ntiles;
+    int32_t *mat = reinterpret_cast<int32_t *>(smem);   // [NT][E] tile counts
+    int32_t *rmat = mat + align4(NT * E);                // [NT][R] tile rank counts (CTA 0)
+    int32_t *base_s = rmat + align4(NT * R);             // [E] rows of expert e before this tile
+    int32_t *cnt_s = base_s + align4(E);                 // [E] expert totals
+    int32_t *seg_s = cnt_s + align4(E);                  // [E+1] segment starts
+    int32_t *wcnt = seg_s + align4(E + 1);               // [W][E]
+    int32_t *ids_s = wcnt + align4(W * E);               // [tile_tokens * k] when a.ids_in_smem
     __shared__ int32_t warp_s[33];
 
-    // Expert totals and exclusive per-tile bases.
-    column_partials(a.tile_cnt, a.ntiles, E, a.scan_parts_e, part);
+    pdl_wait_then_trigger();
+    const int tile = blockIdx.x;
+    const int t0 = tile * a.tile_tokens;
+    const int nt = min(a.tile_tokens, a.T - t0);
+    const int nslots = nt * a.k;
+    const int64_t s0 = (int64_t)t0 * a.k;
+    if (a.ids_in_smem) load_words(ids_s, a.topk_idx + s0, nslots);
+    load_words(mat, a.tile_cnt, NT * E);
+    if (tile == 0) load_words(rmat, a.tile_rank, NT * R);
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t run = 0;
-        for (int p = 0; p < a.scan_parts_e; ++p) {
-            const int32_t v = part[p * E + e];
-            part[p * E + e] = run;
-            run += v;
-        }
-        cnt_s[e] = run;
-    }
-    __syncthreads();
-    for (int item = threadIdx.x; item < partE; item += blockDim.x) {
-        const int e = item % E;
-        const int p = item / E;
-        const int lo = (int)((int64_t)p * a.ntiles / a.scan_parts_e);
-        const int hi = (int)((int64_t)(p + 1) * a.ntiles / a.scan_parts_e);
-        int32_t run = part[item];
-        for (int t = lo; t < hi; ++t) {
-            int32_t *cell = a.tile_cnt + (int64_t)t * E + e;
-            const int32_t v = *cell;
-            *cell = run;
-            run += v;
-        }
-    }
 
-    // Segment offsets: exclusive scan of the segment sizes over experts.
+    // Tile base and total of every expert.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t pre = 0, tot = 0;
+        for (int t = 0; t < NT; ++t) {
+            const int32_t v = mat[t * E + e];
+            pre += (t < tile) ? v : 0;
+            tot += v;
+        }
+        base_s[e] = pre;
+        cnt_s[e] = tot;
+    }
+    __syncthreads();
+
+    // Segment starts: exclusive scan of the segment sizes over experts.
     int32_t carry = 0;
+    bool over = false;
     for (int base = 0; base < E; base += blockDim.x) {
         const int e = base + threadIdx.x;
         int32_t sz = 0;
@@ -187,7 +210,7 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a)
             const int32_t c = cnt_s[e];
             if (a.capacity > 0) {
                 sz = a.capacity;
-                if (c > a.capacity) atomicOr(a.err, kErrCapacity);
+                over |= c > a.capacity;
             } else {
                 sz = (c + a.align - 1) / a.align * a.align;
             }
@@ -198,78 +221,55 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a)
         carry += total;
     }
     if (threadIdx.x == 0) seg_s[E] = carry;
-    __syncthreads();
+    over = __syncthreads_or(over);
 
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.seg[e] = seg_s[e];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        a.cnt[e] = cnt_s[e];
-        if (a.out_cnt != nullptr) a.out_cnt[e] = cnt_s[e];
-    }
-    for (int r = threadIdx.x; r <= R; r += blockDim.x) a.rank_off[r] = seg_s[r * a.epr];
-    __syncthreads();  // part[] is reused below
-
-    // Rank token counts.
-    column_partials(a.tile_rank, a.ntiles, R, a.scan_parts_r, part);
-    __syncthreads();
-    if (a.out_rank_tok != nullptr) {
-        for (int r = threadIdx.x; r < R; r += blockDim.x) {
-            int32_t s = 0;
-            for (int p = 0; p < a.scan_parts_r; ++p) s += part[p * R + r];
-            a.out_rank_tok[r] = s;
+    if (tile == 0) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) a.seg[e] = seg_s[e];
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            a.cnt[e] = cnt_s[e];
+            if (a.out_cnt != nullptr) a.out_cnt[e] = cnt_s[e];
         }
+        for (int r = threadIdx.x; r <= R; r += blockDim.x) a.rank_off[r] = seg_s[r * a.epr];
+        if (a.out_rank_tok != nullptr) {
+            for (int r = threadIdx.x; r < R; r += blockDim.x) {
+                int32_t s = 0;
+                for (int t = 0; t < NT; ++t) s += rmat[t * R + r];
+                a.out_rank_tok[r] = s;
+            }
+        }
+        uint32_t bad = 0u;
+        for (int t = threadIdx.x; t < NT; t += blockDim.x) bad |= __ldg(a.tile_err + t);
+        bad = __syncthreads_or(bad != 0u) ? kErrBadExpertId : 0u;
+        // The layout (re)initialises the handle's error word.
+        if (threadIdx.x == 0) *a.err = bad | (over ? kErrCapacity : 0u);
     }
 
-    // Padding rows get src_idx = -1: the tail of every segment past its
-    // (capacity-clamped) count, and the rows past the last segment.
+    // Padding rows get src_idx = -1: each CTA takes the experts e with
+    // e % ntiles == tile and a share of the rows past the last segment.
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
-    for (int e = warp; e < E; e += nwarps) {
+    for (int e = tile + NT * warp; e < E; e += NT * nwarps) {
         int32_t used = cnt_s[e];
         if (a.capacity > 0) used = min(used, a.capacity);
         for (int64_t row = (int64_t)seg_s[e] + used + lane; row < seg_s[e + 1]; row += 32)
             a.src_idx[row] = -1;
     }
-    for (int64_t row = (int64_t)seg_s[E] + threadIdx.x; row < a.n_rows; row += blockDim.x)
+    for (int64_t row = (int64_t)seg_s[E] + (int64_t)tile * blockDim.x + threadIdx.x; row < a.n_rows;
+         row += (int64_t)NT * blockDim.x)
         a.src_idx[row] = -1;
-}
 
-// ---------------------------------------------------------------------------
-// 3. positions
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int E = a.E;
-    const int W = a.pos_warps;
-    int32_t *base_s = reinterpret_cast<int32_t *>(smem);  // [E] tile base inside each expert
-    int32_t *seg_s = base_s + E;                          // [E]
-    int32_t *wcnt = seg_s + E;                            // [W][E]
-
-    const int tile = blockIdx.x;
-    const int t0 = tile * a.tile_tokens;
-    const int nt = min(a.tile_tokens, a.T - t0);
-    const int nslots = nt * a.k;
-    const int64_t s0 = (int64_t)t0 * a.k;
-
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        base_s[e] = a.tile_cnt[(int64_t)tile * E + e];
-        seg_s[e] = a.seg[e];
-    }
-    for (int i = threadIdx.x; i < W * E; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
+    // Positions of this tile's slots.
     const int lo = (int)((int64_t)warp * nslots / W);
     const int hi = (int)((int64_t)(warp + 1) * nslots / W);
     const unsigned lt_mask = (1u << lane) - 1u;
     int32_t *my = wcnt + warp * E;
 
-    // A: slots of this warp's contiguous range, counted per expert.
+    // A: per-expert slot counts of this warp's contiguous range.
     if (warp < W) {
         for (int b = lo; b < hi; b += 32) {
             const int s = b + lane;
-            const int e = (s < hi) ? load_id(a, s0 + s, false) : -1;
+            const int e = (s < hi) ? tile_id(a, ids_s, s0, s) : -1;
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
             __syncwarp();
@@ -288,11 +288,11 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     }
     __syncthreads();
 
-    // C: ranks in slot order; position = segment start + rank inside the expert.
+    // C: rank inside the expert in slot order; position = segment start + rank.
     if (warp < W) {
         for (int b = lo; b < hi; b += 32) {
             const int s = b + lane;
-            const int e = (s < hi) ? load_id(a, s0 + s, false) : -1;
+            const int e = (s < hi) ? tile_id(a, ids_s, s0, s) : -1;
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             int32_t rel = 0;
             if (e >= 0) rel = my[e] + __popc(peers & lt_mask);
@@ -311,39 +311,52 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     }
 }
 
+// T == 0: no tiles; one CTA writes the (empty or padded) segments, zero
+// counts, -1 over every row and a clear error word.
+__global__ void __launch_bounds__(kPosThreads) layout_empty_kernel(LayoutArgs a) {
+    pdl_wait_then_trigger();
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x)
+        a.seg[e] = a.capacity > 0 ? e * a.capacity : 0;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        a.cnt[e] = 0;
+        if (a.out_cnt != nullptr) a.out_cnt[e] = 0;
+    }
+    for (int r = threadIdx.x; r <= a.R; r += blockDim.x)
+        a.rank_off[r] = a.capacity > 0 ? r * a.epr * a.capacity : 0;
+    if (a.out_rank_tok != nullptr)
+        for (int r = threadIdx.x; r < a.R; r += blockDim.x) a.out_rank_tok[r] = 0;
+    for (int64_t row = threadIdx.x; row < a.n_rows; row += blockDim.x) a.src_idx[row] = -1;
+    if (threadIdx.x == 0) *a.err = 0u;
+}
+
 }  // namespace
 
+size_t layout_count_smem(const LayoutArgs &a) {
+    return (size_t)(a.E + a.R + align4(a.sub_tokens * ((a.R + 31) / 32)) +
+                    (a.ids_in_smem ? a.tile_tokens * a.k : 0)) * 4;
+}
+
+size_t layout_pos_smem(const LayoutArgs &a) {
+    return (size_t)layout_pos_smem_words(a.ntiles, a.E, a.R, a.pos_warps,
+                                         a.ids_in_smem ? a.tile_tokens * a.k : 0) * 4;
+}
+
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s) {
-    const size_t count_smem = (size_t)(a.E + a.R) * 4 + (size_t)a.sub_tokens * a.R * 4;
-    const size_t scan_smem =
-        (size_t)(max(a.scan_parts_e * a.E, a.scan_parts_r * a.R) + a.E + a.E + 1) * 4;
-    const size_t pos_smem = (size_t)(2 + a.pos_warps) * a.E * 4;
     cudaError_t err;
+    if (a.ntiles == 0) return launch_kernel(layout_empty_kernel, 1, kPosThreads, 0, s, a);
+    const size_t count_smem = layout_count_smem(a);
+    const size_t pos_smem = layout_pos_smem(a);
     if (count_smem > 48 * 1024 &&
         (err = cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)count_smem)) != cudaSuccess)
-        return err;
-    if (scan_smem > 48 * 1024 &&
-        (err = cudaFuncSetAttribute(layout_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)scan_smem)) != cudaSuccess)
         return err;
     if (pos_smem > 48 * 1024 &&
         (err = cudaFuncSetAttribute(layout_pos_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)pos_smem)) != cudaSuccess)
         return err;
-    if (a.ntiles > 0) {
-        layout_count_kernel<<<a.ntiles, kCountThreads, count_smem, s>>>(a);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    }
-    // The scan also runs for T == 0: it writes the (empty or padded) segments,
-    // zero counts and the -1 fill of every row.
-    layout_scan_kernel<<<1, kScanThreads, scan_smem, s>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (a.ntiles > 0) {
-        layout_pos_kernel<<<a.ntiles, kPosThreads, pos_smem, s>>>(a);
-        return cudaGetLastError();
-    }
-    return cudaSuccess;
+    if ((err = launch_kernel(layout_count_kernel, a.ntiles, kCountThreads, count_smem, s, a)) != cudaSuccess)
+        return err;
+    return launch_kernel(layout_pos_kernel, a.ntiles, kPosThreads, pos_smem, s, a);
 }
 
 }  // namespace ep

@@ -19,9 +19,9 @@
 // calls on a device share the array, so two calls whose work overlaps on the
 // GPU (different streams, no ordering between them) race on it; calls on one
 // stream are ordered and safe.  Nothing in it needs to start at zero: the
-// count kernel overwrites every tile entry it uses and the error word is
-// cleared by this call.
-#include <algorithm>
+// count kernel overwrites every tile entry the position kernel reads, and the
+// position kernel (or, for T == 0, the empty-layout kernel) overwrites the
+// error word.
 #include <mutex>
 
 #include "ep_internal.cuh"
@@ -83,16 +83,16 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
         return EP_ERR_INVALID_ARG;
 
     // Same tile geometry as ep_layout.
-    int tile_tokens = 128;
-    if ((T + tile_tokens - 1) / tile_tokens > 512)
-        tile_tokens = ((T + 511) / 512 + 31) / 32 * 32;
-    const int ntiles = (T + tile_tokens - 1) / tile_tokens;
+    const LayoutGeometry geo = layout_geometry(T, k, E, R);
+    const int ntiles = geo.ntiles;
 
-    // Scratch words: tile_cnt, tile_rank, per-expert counts, error word.
-    const size_t w_tcnt = (size_t)ntiles * E;
-    const size_t w_trank = (size_t)ntiles * R;
-    const size_t w_cnt = (size_t)E;
-    const size_t need = w_tcnt + w_trank + w_cnt + 1;
+    // Scratch words (16-byte aligned blocks): tile_cnt, tile_rank, per-expert
+    // counts, per-tile bad-id flags, error word.
+    const size_t w_tcnt = (size_t)align4(ntiles * E);
+    const size_t w_trank = (size_t)align4(ntiles * R);
+    const size_t w_cnt = (size_t)align4(E);
+    const size_t w_terr = (size_t)align4(ntiles);
+    const size_t need = w_tcnt + w_trank + w_cnt + w_terr + 1;
     if (need > (size_t)EP_NOALLOC_SCRATCH_WORDS) return EP_ERR_SCRATCH_LIMIT;
 
     int dev = 0;
@@ -108,12 +108,11 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
     LayoutArgs a{};
     a.topk_idx = topk_idx;
     a.T = T; a.k = k; a.E = E; a.R = R; a.epr = E / R; a.align = A; a.capacity = C;
-    a.tile_tokens = tile_tokens;
+    a.tile_tokens = geo.tile_tokens;
     a.ntiles = ntiles;
-    a.sub_tokens = std::max(1, std::min(tile_tokens, 4096 / R));
-    a.scan_parts_e = std::max(1, std::min(std::max(ntiles, 1), 1024 / E));
-    a.scan_parts_r = std::max(1, std::min(std::max(ntiles, 1), 1024 / R));
-    a.pos_warps = std::min(8, std::max(1, 12288 / E));
+    a.sub_tokens = geo.sub_tokens;
+    a.pos_warps = geo.pos_warps;
+    a.ids_in_smem = geo.ids_in_smem;
     a.n_rows = (int64_t)n_rows;
     a.pos = pos;
     a.src_idx = src_idx;
@@ -122,13 +121,13 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
     a.tile_cnt = scratch;
     a.tile_rank = scratch + w_tcnt;
     a.cnt = scratch + w_tcnt + w_trank;
+    a.tile_err = reinterpret_cast<uint32_t *>(scratch + w_tcnt + w_trank + w_cnt);
     a.err = error_word != nullptr ? error_word
-                                  : reinterpret_cast<uint32_t *>(scratch + w_tcnt + w_trank + w_cnt);
+                                  : reinterpret_cast<uint32_t *>(scratch + w_tcnt + w_trank + w_cnt + w_terr);
     a.out_cnt = out_cnt;
     a.out_rank_tok = out_rank_tok;
     a.out_in_rank = out_in_rank;
 
-    e = cudaMemsetAsync(a.err, 0, 4, stream);
-    if (e == cudaSuccess) e = launch_layout(a, stream);
-    return status_of(e);
+    // The layout kernels overwrite the error word; nothing else needs clearing.
+    return status_of(launch_layout(a, stream));
 }

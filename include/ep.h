@@ -45,7 +45,7 @@
  *     synchronises.
  *   - Argument errors are detected on the host and returned at once with
  *     nothing enqueued.  Data errors found on the device (an id outside
- *     [-1, E), a padded expert over capacity, a timed-out wait) set the
+ *     [-1, E), a padded expert over capacity) set the
  *     handle's device error word instead; the outputs of that call are then
  *     unspecified but every device write stays inside the buffers described
  *     here.  ep_handle_check() reports the word.  No call traps, aborts or
@@ -78,7 +78,7 @@ typedef enum ep_status {
     EP_ERR_CAPACITY = 3,      /* padded mode: an expert received more than `capacity` tokens */
     EP_ERR_CUDA = 4,          /* a CUDA runtime call failed */
     EP_ERR_OOM = 5,           /* device allocation failed */
-    EP_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up */
+    EP_ERR_TIMEOUT = 6,       /* reserved: a bounded device-side wait gave up (no kernel waits today) */
     EP_ERR_NO_DEVICE = 7,     /* no CUDA device, or the device is not sm_100 */
     EP_ERR_SCRATCH_LIMIT = 8  /* ep_layout_noalloc: the problem needs more than its fixed scratch */
 } ep_status;
@@ -106,7 +106,9 @@ size_t ep_max_recv_rows(int num_tokens, int num_topk, int num_experts,
  *   capacity: 0 for packed mode, else rows per expert (a multiple of expert_alignment).
  * On success *out_handle receives a handle that the caller frees with
  * ep_handle_free().  The handle's device memory is allocated stream-ordered
- * on `stream` (cudaMallocAsync).  T == 0 is allowed (empty handle). */
+ * on `stream` from a memory pool the library keeps per device (memory freed by
+ * ep_handle_free returns to that pool for the next layout, not to the
+ * driver).  T == 0 is allowed (empty handle). */
 ep_status ep_layout(const int32_t *topk_idx, int num_tokens, int num_topk,
                     int num_experts, int num_ranks, int expert_alignment, int capacity,
                     int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
@@ -176,9 +178,9 @@ ep_status ep_handle_counts_host(const ep_handle *handle, int32_t *host_counts,
 ep_status ep_handle_check(const ep_handle *handle, ep_stream_t stream);
 
 /* Size, in 32-bit words, of the fixed device scratch array ep_layout_noalloc
- * uses (1 MiB).  Every GPU that loads the library holds it until the process
- * exits. */
-#define EP_NOALLOC_SCRATCH_WORDS (1 << 18)
+ * uses (128 KiB).  Every GPU that loads the library holds it until the
+ * process exits. */
+#define EP_NOALLOC_SCRATCH_WORDS (1 << 15)
 
 /* ep_layout_noalloc -- the routing layout of ep_layout, for callers that
  * cannot allocate device memory.  The pages have no counterpart: DeepEP's
@@ -202,8 +204,11 @@ ep_status ep_handle_check(const ep_handle *handle, ep_stream_t stream);
  * Allocates nothing: no cudaMalloc / cudaMallocAsync / cudaFree and no
  * allocating library routine.  Its only device memory besides the caller's
  * buffers is a fixed scratch array of EP_NOALLOC_SCRATCH_WORDS words inside
- * the library; a problem whose per-tile count matrices need more
- * (about ceil(T/128) * (E + R) + E + 1 words) is rejected with
+ * the library; a problem that needs more is rejected.  The need is
+ * align4(tiles*E) + align4(tiles*R) + align4(E) + align4(tiles) + 1 words,
+ * with tiles = ceil(T / tile) and tile = 128 tokens, doubled until
+ * tiles*(E + R) <= 24576: every problem with E + R >= 8 fits; with very few
+ * experts and millions of tokens the per-tile flags can exceed it is rejected with
  * EP_ERR_SCRATCH_LIMIT before anything is enqueued.  The first call on a
  * device looks up the array's device address (once per device, with that
  * device current); make that first call before any stream capture.  All calls

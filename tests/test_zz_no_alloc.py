@@ -70,7 +70,9 @@ def test_noalloc_matches_layout_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    T, k, E, R = 8192, 1, 4096, 4096   # 64 tiles x 8192 words > 2^18
+    # One expert, one rank: 12288 tiles of 128 tokens; the per-tile words
+    # (2 count words + 1 flag word per tile) exceed the 2^15-word scratch.
+    T, k, E, R = 12288 * 128, 1, 1, 1
     idx = torch.zeros(T, k, dtype=torch.int32, device=DEV)
     rows = ep.ep_max_recv_rows(T, k, E)
     b = buffers(T, k, E, R, rows)
