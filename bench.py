@@ -50,8 +50,8 @@ HBM_FALLBACK_GBS = 6650.0
 # kernel source it was taken on (stale -> reported as null).
 NCU_TRAFFIC = {
     # one "ncu --set full" capture of one launch each on the metric workload
-    ("group_limited", "combine"): {"sha": "bf4a5eb031b55673", "bytes": 940059648 + 73684224},
-    ("group_limited", "dispatch"): {"sha": "8dcb1a902f506325", "bytes": 117851648 + 426448384},
+    ("group_limited", "combine"): {"sha": "e4aaa5203a4c74cf", "bytes": 940057856 + 73635328},
+    ("group_limited", "dispatch"): {"sha": "23a3a09c311a730d", "bytes": 117871104 + 427218944},
 }
 
 

@@ -107,7 +107,12 @@ constexpr int kLayoutMatWords = 24576;
 struct LayoutGeometry {
     int tile_tokens, ntiles, sub_tokens, pos_warps;
     bool ids_in_smem;  // the position kernel stages the tile's ids in shared memory
+    bool small;        // the whole layout fits one CTA (layout_small_kernel)
 };
+// Shared-memory words of the one-CTA layout (32 warps).
+inline int layout_small_smem_words(int T, int k, int E, int R) {
+    return align4(T * k) + align4(E) + align4(E + 1) + align4(R) + 32 * (E + 1) + T * ((R + 31) / 32);
+}
 // Shared-memory words of the position kernel.
 inline int layout_pos_smem_words(int ntiles, int E, int R, int pos_warps, int id_words) {
     return align4(ntiles * E) + align4(ntiles * R) + 2 * align4(E) + align4(E + 1) +
@@ -126,6 +131,8 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R) {
     const int64_t id_words = (int64_t)g.tile_tokens * k;
     g.ids_in_smem = id_words <= 8192 &&
                     layout_pos_smem_words(g.ntiles, E, R, g.pos_warps, (int)id_words) <= 50000;
+    g.small = T > 0 && (int64_t)T * k <= 8192 && E <= 512 &&
+              layout_small_smem_words(T, k, E, R) <= 40000;
     return g;
 }
 
@@ -133,7 +140,7 @@ struct LayoutArgs {
     const int32_t *topk_idx;
     int T, k, E, R, epr, align, capacity;
     int tile_tokens, ntiles, sub_tokens, pos_warps;
-    bool ids_in_smem;
+    bool ids_in_smem, small;
     int64_t n_rows;
     int32_t *pos, *src_idx, *seg, *rank_off, *cnt, *tile_cnt, *tile_rank;
     uint32_t *tile_err, *err;
@@ -166,6 +173,7 @@ struct CombineArgs {
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 size_t layout_count_smem(const LayoutArgs &a);
+size_t layout_small_smem(const LayoutArgs &a);
 size_t layout_pos_smem(const LayoutArgs &a);
 cudaError_t launch_dispatch(const DispatchArgs &a, bool fp8, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);

@@ -21,6 +21,8 @@
 //      and a prefix over its warps, and writes pos[t][j] and src_idx[row].
 //      CTA 0 publishes counts, segments, rank slices, rank counts and the
 //      error word; the -1 fill of padding rows is spread over all CTAs.
+#include <atomic>
+
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -311,6 +313,164 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     }
 }
 
+// dst[0, n) = -1 by the calling CTA, 16-byte stores where aligned.
+__device__ __forceinline__ void fill_minus_one(int32_t *dst, int64_t n) {
+    int64_t head = (int64_t)((16 - (reinterpret_cast<uintptr_t>(dst) & 15u)) & 15u) / 4;
+    if (head > n) head = n;
+    for (int64_t i = threadIdx.x; i < head; i += blockDim.x) dst[i] = -1;
+    const int64_t n4 = (n - head) >> 2;
+    int4 *d4 = reinterpret_cast<int4 *>(dst + head);
+    for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) d4[i] = make_int4(-1, -1, -1, -1);
+    for (int64_t i = head + (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) dst[i] = -1;
+}
+
+// ---------------------------------------------------------------------------
+// Small problems: the whole layout in one CTA of 1024 threads
+// ---------------------------------------------------------------------------
+// With at most 8192 slots, one CTA holds every id, the expert histogram, the
+// per-warp counts and the rank bitmasks in shared memory, so counts, segments
+// and positions need no second kernel and no count matrices in global memory.
+// The 32 warps own contiguous slot ranges; ranks inside an expert come from
+// __match_any_sync + popc plus a prefix over the warps, as in the tiled path.
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+
+__global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    pdl_wait_then_trigger();
+    const int E = a.E, R = a.R;
+    const int RW = (R + 31) >> 5;
+    const int nslots = a.T * a.k;
+    int32_t *ids_s = reinterpret_cast<int32_t *>(smem);      // [nslots]
+    int32_t *cnt_s = ids_s + align4(nslots);                   // [E]
+    int32_t *seg_s = cnt_s + align4(E);                        // [E+1]
+    int32_t *rcnt_s = seg_s + align4(E + 1);                   // [R]
+    // Per-warp counts, rows padded to an odd stride (E + 1 words) so that the
+    // warp-parallel prefix below (lane = warp index) hits 32 different banks.
+    const int ldw = E + 1;
+    int32_t *wcnt = rcnt_s + align4(R);                        // [32][E + 1]
+    uint32_t *mask_s = reinterpret_cast<uint32_t *>(wcnt + kSmallWarps * ldw);  // [T][RW]
+    __shared__ int32_t warp_s[33];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    load_words(ids_s, a.topk_idx, nslots);
+    for (int i = threadIdx.x; i < R; i += blockDim.x) rcnt_s[i] = 0;
+    for (int i = threadIdx.x; i < kSmallWarps * ldw; i += blockDim.x) wcnt[i] = 0;
+    for (int i = threadIdx.x; i < a.T * RW; i += blockDim.x) mask_s[i] = 0u;
+    __syncthreads();
+
+    // One pass over the slots: warp w owns the contiguous range [lo, hi) and
+    // counts it per expert with __match_any_sync (leader lane adds popc);
+    // every valid slot also sets its token's rank bit (the slot that sets it
+    // counts the token for that rank).
+    const int lo = (int)((int64_t)warp * nslots / kSmallWarps);
+    const int hi = (int)((int64_t)(warp + 1) * nslots / kSmallWarps);
+    int32_t *my = wcnt + warp * ldw;
+    int bad = 0;
+    for (int b = lo; b < hi; b += 32) {
+        const int sidx = b + lane;
+        int e = -1;
+        if (sidx < hi) {
+            e = ids_s[sidx];
+            if (e < -1 || e >= E) {
+                bad = 1;
+                e = -1;
+                ids_s[sidx] = -1;  // treated as unused from here on
+            }
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0) {
+            if (lane == __ffs(peers) - 1) my[e] += __popc(peers);
+            const int r = e / a.epr;
+            const uint32_t bit = 1u << (r & 31);
+            if (!(atomicOr(&mask_s[(sidx / a.k) * RW + (r >> 5)], bit) & bit)) atomicAdd(&rcnt_s[r], 1);
+        }
+        __syncwarp();
+    }
+    bad = __syncthreads_or(bad);
+
+    // Exclusive prefix over the 32 warps of every expert (one warp per expert,
+    // lane = warp index) and the expert totals.
+    for (int e = warp; e < E; e += kSmallWarps) {
+        const int32_t v = wcnt[lane * ldw + e];
+        int32_t incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t n = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += n;
+        }
+        wcnt[lane * ldw + e] = incl - v;
+        if (lane == 31) cnt_s[e] = incl;
+    }
+    __syncthreads();
+
+    // Segments.
+    int32_t carry = 0;
+    bool over = false;
+    for (int base = 0; base < E; base += blockDim.x) {
+        const int e = base + threadIdx.x;
+        int32_t sz = 0;
+        if (e < E) {
+            const int32_t c = cnt_s[e];
+            if (a.capacity > 0) {
+                sz = a.capacity;
+                over |= c > a.capacity;
+            } else {
+                sz = (c + a.align - 1) / a.align * a.align;
+            }
+        }
+        int32_t total;
+        const int32_t excl = block_exclusive_scan(sz, &total, warp_s);
+        if (e < E) seg_s[e] = carry + excl;
+        carry += total;
+    }
+    if (threadIdx.x == 0) seg_s[E] = carry;
+    over = __syncthreads_or(over);
+
+    // Publish counts, segments, rank slices and counts, the error word, the
+    // token-in-rank rows; every row of src_idx starts as padding (-1).
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.seg[e] = seg_s[e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        a.cnt[e] = cnt_s[e];
+        if (a.out_cnt != nullptr) a.out_cnt[e] = cnt_s[e];
+    }
+    for (int r = threadIdx.x; r <= R; r += blockDim.x) a.rank_off[r] = seg_s[r * a.epr];
+    if (a.out_rank_tok != nullptr)
+        for (int r = threadIdx.x; r < R; r += blockDim.x) a.out_rank_tok[r] = rcnt_s[r];
+    if (threadIdx.x == 0) *a.err = (bad ? kErrBadExpertId : 0u) | (over ? kErrCapacity : 0u);
+    if (a.out_in_rank != nullptr) {
+        for (int i = threadIdx.x; i < a.T * R; i += blockDim.x) {
+            const int t = i / R;
+            const int r = i - t * R;
+            a.out_in_rank[i] = (uint8_t)((mask_s[t * RW + (r >> 5)] >> (r & 31)) & 1u);
+        }
+    }
+    fill_minus_one(a.src_idx, a.n_rows);
+    __syncthreads();  // orders the -1 fill before the valid rows below
+
+    // Positions: rank inside the expert in slot order.
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int b = lo; b < hi; b += 32) {
+        const int sidx = b + lane;
+        const int e = (sidx < hi) ? ids_s[sidx] : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        int32_t rel = 0;
+        if (e >= 0) rel = my[e] + __popc(peers & lt_mask);
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+        __syncwarp();
+        if (sidx < hi) {
+            int32_t p = -1;
+            if (e >= 0 && (a.capacity == 0 || rel < a.capacity)) {
+                p = seg_s[e] + rel;
+                a.src_idx[p] = sidx / a.k;
+            }
+            a.pos[sidx] = p;
+        }
+    }
+}
+
 // T == 0: no tiles; one CTA writes the (empty or padded) segments, zero
 // counts, -1 over every row and a clear error word.
 __global__ void __launch_bounds__(kPosThreads) layout_empty_kernel(LayoutArgs a) {
@@ -331,6 +491,10 @@ __global__ void __launch_bounds__(kPosThreads) layout_empty_kernel(LayoutArgs a)
 
 }  // namespace
 
+size_t layout_small_smem(const LayoutArgs &a) {
+    return (size_t)layout_small_smem_words(a.T, a.k, a.E, a.R) * 4;
+}
+
 size_t layout_count_smem(const LayoutArgs &a) {
     return (size_t)(a.E + a.R + align4(a.sub_tokens * ((a.R + 31) / 32)) +
                     (a.ids_in_smem ? a.tile_tokens * a.k : 0)) * 4;
@@ -341,19 +505,36 @@ size_t layout_pos_smem(const LayoutArgs &a) {
                                          a.ids_in_smem ? a.tile_tokens * a.k : 0) * 4;
 }
 
+// Raise a kernel's dynamic shared-memory limit when a launch needs more than
+// the default (48 KiB including static shared memory; 32 KiB leaves room).
+// Cached per device: the attribute is set once per size increase.
+template <typename Kernel>
+cudaError_t ensure_dyn_smem(Kernel kernel, size_t bytes, std::atomic<int> *cache) {
+    if (bytes <= 32 * 1024) return cudaSuccess;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (cache[dev].load(std::memory_order_relaxed) >= (int)bytes) return cudaSuccess;
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (err == cudaSuccess) cache[dev].store((int)bytes, std::memory_order_relaxed);
+    return err;
+}
+
+std::atomic<int> g_smem_small[64], g_smem_count[64], g_smem_pos[64];
+
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s) {
     cudaError_t err;
     if (a.ntiles == 0) return launch_kernel(layout_empty_kernel, 1, kPosThreads, 0, s, a);
+    if (a.small) {
+        const size_t smem = layout_small_smem(a);
+        if ((err = ensure_dyn_smem(layout_small_kernel, smem, g_smem_small)) != cudaSuccess) return err;
+        return launch_kernel(layout_small_kernel, 1, kSmallThreads, smem, s, a);
+    }
     const size_t count_smem = layout_count_smem(a);
     const size_t pos_smem = layout_pos_smem(a);
-    if (count_smem > 48 * 1024 &&
-        (err = cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)count_smem)) != cudaSuccess)
-        return err;
-    if (pos_smem > 48 * 1024 &&
-        (err = cudaFuncSetAttribute(layout_pos_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)pos_smem)) != cudaSuccess)
-        return err;
+    if ((err = ensure_dyn_smem(layout_count_kernel, count_smem, g_smem_count)) != cudaSuccess) return err;
+    if ((err = ensure_dyn_smem(layout_pos_kernel, pos_smem, g_smem_pos)) != cudaSuccess) return err;
     if ((err = launch_kernel(layout_count_kernel, a.ntiles, kCountThreads, count_smem, s, a)) != cudaSuccess)
         return err;
     return launch_kernel(layout_pos_kernel, a.ntiles, kPosThreads, pos_smem, s, a);

@@ -113,6 +113,7 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
     a.sub_tokens = geo.sub_tokens;
     a.pos_warps = geo.pos_warps;
     a.ids_in_smem = geo.ids_in_smem;
+    a.small = geo.small;
     a.n_rows = (int64_t)n_rows;
     a.pos = pos;
     a.src_idx = src_idx;

@@ -85,6 +85,9 @@ LAYOUT_EDGE = [
     (70000, 2, 64, 16, 1, 0, -1),     # > 512 tiles of 128: larger tiles
     (64, 32, 4096, 4096, 1, 0, -1),   # maximum k, E, R
     (2048, 6, 96, 12, 8, 0, -1),      # E not a power of two
+    (5000, 2, 16, 4, 1, 1024, 0),     # padded, tiled path (more than 8192 slots)
+    (8193, 1, 8, 2, 1, 0, -1),        # one slot past the one-CTA limit
+    (8192, 1, 8, 2, 1, 0, -1),        # exactly at the one-CTA limit
 ]
 
 
@@ -118,6 +121,20 @@ def test_layout_bad_expert_id_reported():
     # the valid slots still get a consistent layout; the bad ones none
     pos = res.handle.export()["pos"].cpu().numpy()
     assert pos[1, 1] == -1 and pos[2, 0] == -1
+
+
+def test_layout_errors_on_tiled_path():
+    g = torch.Generator().manual_seed(5)
+    idx = torch.randint(0, 16, (4096, 4), generator=g, dtype=torch.int32)
+    idx[1000, 2] = 16
+    res = ep.ep_layout(idx.to(DEV), 16, 4)
+    assert res.handle.check() == ep.EP_ERR_BAD_EXPERT_ID
+    assert res.handle.export()["pos"].cpu().numpy()[1000, 2] == -1
+    over = torch.zeros(9000, 1, dtype=torch.int32)
+    res = ep.ep_layout(over.to(DEV), 4, 2, 1, 4)
+    assert res.handle.check() == ep.EP_ERR_CAPACITY
+    pos = res.handle.export()["pos"].cpu().numpy().ravel()
+    assert pos[:4].tolist() == [0, 1, 2, 3] and (pos[4:] == -1).all()
 
 
 def test_layout_capacity_overflow_reported():
