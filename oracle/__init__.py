@@ -67,6 +67,8 @@ def lib():
         L.oracle_quantize_group.restype = None
         L.oracle_combine.argtypes = [P, i64, i32, P, P, i32, i32, P]
         L.oracle_combine.restype = i32
+        L.oracle_combine_backward.argtypes = [P, P, i64, i32, P, P, i32, i32, P, P]
+        L.oracle_combine_backward.restype = i32
         _LIB = L
     return _LIB
 
@@ -221,6 +223,31 @@ def combine(y, w: np.ndarray, pos: np.ndarray) -> np.ndarray:
     if st != OR_OK:
         raise OracleError(st, "oracle_combine")
     return out
+
+
+def dispatch_backward(grad_recv, pos: np.ndarray) -> np.ndarray:
+    """Gradient of x from the gradients of the receive rows: the combine with
+    every weight 1 (uint16 bf16 bits [T, H])."""
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    return combine(grad_recv, np.ones(pos.shape, np.float32), pos)
+
+
+def combine_backward(grad_out, y, w: np.ndarray, pos: np.ndarray):
+    """Returns (grad_y uint16 [n_rows, H], rows never written are 0;
+    grad_w float64 [T, k])."""
+    gb = _u16(grad_out)
+    yb = _u16(y)
+    n_rows, H = yb.shape
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    T, k = pos.shape
+    grad_y = np.zeros((n_rows, H), np.uint16)
+    grad_w = np.zeros((T, k), np.float64)
+    st = lib().oracle_combine_backward(_ptr(gb), _ptr(yb), n_rows, H, _ptr(w), _ptr(pos), T, k,
+                                       _ptr(grad_y), _ptr(grad_w))
+    if st != OR_OK:
+        raise OracleError(st, "oracle_combine_backward")
+    return grad_y, grad_w
 
 
 def bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -418,3 +418,55 @@ int oracle_combine(const uint16_t *y, int64_t n_rows, int H, const float *w,
     }
     return OR_OK;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Backward                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* The pages ("DeepSeek publica DeepEP ...", news.hada.io, "Patrones de uso
+ * en entrenamiento, prefill y decoding"; "DeepEP (DeepEveryParallel)
+ * Documentation", item 10) say that the backward pass of dispatch is carried
+ * out by a combine and the backward pass of combine by a dispatch.  Written
+ * out for this library's forward definitions:
+ *
+ * dispatch backward: the gradient reaching x[t] is the sum of the gradients
+ *   of its k receive rows.  That is the combine definition with every weight
+ *   equal to 1 (oracle_combine with w = 1): bf16_rn of the fp32 chain
+ *   acc = acc + grad_recv[pos[t][j]][i] over valid slots in slot order.
+ *
+ * combine backward, with g = grad_out[t] (bf16):
+ *   grad_y[pos[t][j]][i] = bf16_rn( fp32_rn( w[t][j] * g[i] ) )   (a weighted dispatch)
+ *   grad_w[t][j]         = sum_i g[i] * y[pos[t][j]][i]          (a dot product)
+ *   The dot product is returned exactly enough to grade any fp32 summation
+ *   order: every product of two bf16 values is exact in binary64 and the
+ *   binary64 sum of at most 2^16 of them is within ~1e-12 relative of the
+ *   exact sum.  Slots with pos < 0 get grad_w = 0 and write no row. */
+int oracle_combine_backward(const uint16_t *grad_out, const uint16_t *y, int64_t n_rows, int H,
+                            const float *w, const int32_t *pos, int T, int k, uint16_t *grad_y,
+                            double *grad_w) {
+    if (T < 0 || H < 1 || k < 1) {
+        return OR_ERR_INVALID_ARG;
+    }
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int64_t s = (int64_t)t * k + j;
+            int32_t p = pos[s];
+            if (p < 0) {
+                grad_w[s] = 0.0;
+                continue;
+            }
+            if (p >= n_rows) {
+                return OR_ERR_INVALID_ARG;
+            }
+            double dot = 0.0;
+            for (int i = 0; i < H; ++i) {
+                float g = oracle_bf16_to_f32(grad_out[(int64_t)t * H + i]);
+                float prod = w[s] * g;
+                grad_y[(int64_t)p * H + i] = oracle_f32_to_bf16(prod);
+                dot += (double)g * (double)oracle_bf16_to_f32(y[(int64_t)p * H + i]);
+            }
+            grad_w[s] = dot;
+        }
+    }
+    return OR_OK;
+}
