@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-cpu-baseline] [--no-e2e] [--no-decode]
+                    [--no-backward]
 
 A step is one pass of the whole path over one batch: ep_layout (2 kernels),
 ep_dispatch (FP8 e4m3 or BF16), ep_combine (BF16), all through the C ABI.
@@ -65,6 +66,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-backward", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
 
@@ -509,6 +511,10 @@ def run_ours(args, w):
     if not args.no_decode:
         decode = run_decode_latency(dev, ep)
 
+    backward = None
+    if not args.no_backward:
+        backward = run_backward(w, dev, ep, idx, tw, y, flush_l2)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed)
@@ -521,7 +527,7 @@ def run_ours(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "decode": decode,
+            "decode": decode, "backward": backward,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "wall_s": wall,
             "host_us_per_step": host_s * 1e6,
         }
@@ -609,6 +615,52 @@ def run_decode_latency(dev, ep, steps: int = 100) -> dict:
             "capacity": w.capacity, "steps": steps, "dispatch_us": d_us, "combine_us": c_us,
             "step_us_plain": d_us + c_us, "step_us_graph": total / steps * 1e3,
             "dispatch_bytes": disp_bytes, "combine_bytes": comb_bytes}
+
+
+def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) -> dict:
+    """The backward pair on the step's layout: ep_dispatch_backward (the
+    combine with unit weights) and ep_combine_backward (weighted scatter of
+    grad_out plus the grad_weights dot products), each timed with the L2
+    flushed before every call."""
+    T, H, k = w.T, w.H, w.k
+    res = ep.ep_layout(idx_dev, w.E, w.R, w.align, w.capacity)
+    h = res.handle
+    rows = h.num_recv_rows
+    g = torch.Generator(device=dev).manual_seed(77)
+    grad_recv = torch.randn(rows, H, generator=g, device=dev).to(torch.bfloat16)
+    grad_out = torch.randn(T, H, generator=g, device=dev).to(torch.bfloat16)
+    grad_x = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    grad_y = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+    grad_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        ts = []
+        for i in range(steps + 3):
+            flush_l2()
+            torch.cuda._sleep(GPU_LEAD_CYCLES // 2)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if i >= 3:
+                ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ts) * 1e3
+
+    d_us = timed(lambda: ep.ep_dispatch_backward(h, grad_recv, grad_x))
+    c_us = timed(lambda: ep.ep_combine_backward(h, grad_out, tw_dev, y=y_dev, grad_y=grad_y,
+                                                grad_weights=grad_w))
+    status = h.check()
+    h.free()
+    if status != ep.EP_OK:
+        raise SystemExit("backward: device error %s" % ep.status_str(status))
+    V = int((idx_dev >= 0).sum().item())
+    d_bytes = V * H * 2 + T * k * 4 + T * H * 2
+    c_bytes = T * H * 2 + V * H * 2 + T * k * 8 + V * H * 2 + T * k * 4
+    return {"dispatch_backward": {"us": d_us, "bytes": d_bytes, "gbs": d_bytes / d_us / 1e3},
+            "combine_backward": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3}}
 
 
 def run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y_dev, nbytes, world):

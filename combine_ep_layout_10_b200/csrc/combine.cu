@@ -14,7 +14,9 @@
 // one token, issues all k row loads of a batch before it accumulates (k
 // independent 16-byte loads in flight per thread, read-only non-coherent path
 // without L1 allocation: y is never written during the kernel), then runs the
-// FMA chain in slot order and stores 16 bytes.
+// FMA chain in slot order and stores 16 bytes.  With no weights (w == nullptr)
+// every weight is 1: fmaf(1, y, acc) is the correctly rounded acc + y, which
+// makes the same kernel the backward of dispatch (sum of the k row gradients).
 #include <cuda_bf16.h>
 
 #include "ep_internal.cuh"
@@ -75,7 +77,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
     const int cb = blockIdx.x - t * a.blocks_per_token;
     if (threadIdx.x < a.k) {
         p_s[threadIdx.x] = __ldg(a.pos + (int64_t)t * a.k + threadIdx.x);
-        w_s[threadIdx.x] = __ldg(a.w + (int64_t)t * a.k + threadIdx.x);
+        w_s[threadIdx.x] = a.w != nullptr ? __ldg(a.w + (int64_t)t * a.k + threadIdx.x) : 1.0f;
     }
     __syncthreads();
 

@@ -279,6 +279,54 @@ ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int
     return cuda_status(launch_combine(a, stream));
 }
 
+ep_status ep_dispatch_backward(const ep_handle *h, const void *grad_recv, int H, size_t recv_rows,
+                               void *grad_x, ep_stream_t stream) {
+    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    if (h->T > 0 && (grad_recv == nullptr || grad_x == nullptr || !aligned(grad_recv, 16) || !aligned(grad_x, 16)))
+        return EP_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != h->device) return EP_ERR_INVALID_ARG;
+    CombineArgs a{};
+    a.y = static_cast<const uint8_t *>(grad_recv);
+    a.w = nullptr;  // unit weights
+    a.pos = h->pos;
+    a.out = static_cast<uint8_t *>(grad_x);
+    a.T = h->T; a.k = h->k; a.H = H;
+    a.nvec = H / 8;
+    a.vpt = EP_COMBINE_VPT;
+    a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
+    return cuda_status(launch_combine(a, stream));
+}
+
+ep_status ep_combine_backward(const ep_handle *h, const void *grad_out, const void *y, const float *topk_w,
+                              int H, size_t recv_rows, void *grad_y, float *grad_w, ep_stream_t stream) {
+    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    if (h->T > 0) {
+        if (grad_out == nullptr || topk_w == nullptr || grad_y == nullptr) return EP_ERR_INVALID_ARG;
+        if (!aligned(grad_out, 16) || !aligned(grad_y, 16) || !aligned(topk_w, 4)) return EP_ERR_INVALID_ARG;
+        if (grad_w != nullptr && (y == nullptr || !aligned(y, 16) || !aligned(grad_w, 4))) return EP_ERR_INVALID_ARG;
+    }
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != h->device) return EP_ERR_INVALID_ARG;
+    CombineBwdArgs a{};
+    a.grad_out = static_cast<const uint8_t *>(grad_out);
+    a.y = static_cast<const uint8_t *>(y);
+    a.w = topk_w;
+    a.pos = h->pos;
+    a.grad_y = static_cast<uint8_t *>(grad_y);
+    a.grad_w = grad_w;
+    a.T = h->T; a.k = h->k; a.H = H;
+    return cuda_status(launch_combine_backward(a, stream));
+}
+
 void ep_handle_free(ep_handle *h) {
     if (h == nullptr) return;
     if (h->block != nullptr) {

@@ -27,6 +27,15 @@
 #define EP_COMBINE_STREAM_STORE 0
 #endif
 
+#ifndef EP_BWD_BATCH              // combine backward: y rows loaded ahead per batch of slots
+#define EP_BWD_BATCH 8
+#endif
+#ifndef EP_BWD_MAX_THREADS        // combine backward: threads per block (upper bound)
+#define EP_BWD_MAX_THREADS 128
+#endif
+#ifndef EP_BWD_MIN_BLOCKS         // combine backward: resident blocks per SM to plan registers for
+#define EP_BWD_MIN_BLOCKS 4
+#endif
 #ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
 #define EP_USE_PDL 1
 #endif
@@ -161,13 +170,23 @@ struct DispatchArgs {
 
 struct CombineArgs {
     const uint8_t *y;        // bf16 [rows, H]
-    const float *w;          // [T, k]
+    const float *w;          // [T, k], or nullptr for unit weights (dispatch backward)
     const int32_t *pos;      // [T, k]
     uint8_t *out;            // bf16 [T, H]
     int T, k, H;
     int nvec;                // H / 8 (16-byte vectors per row)
     int vpt;                 // vectors per thread: 1, 2 or 4
     int blocks_per_token;    // ceil(nvec / (128 * vpt))
+};
+
+struct CombineBwdArgs {
+    const uint8_t *grad_out; // bf16 [T, H]
+    const uint8_t *y;        // bf16 [rows, H] (only read when grad_w != nullptr)
+    const float *w;          // [T, k]
+    const int32_t *pos;      // [T, k]
+    uint8_t *grad_y;         // bf16 [rows, H]
+    float *grad_w;           // [T, k] or nullptr
+    int T, k, H;
 };
 
 // Launchers (return the cudaGetLastError() of the launch).
@@ -177,6 +196,7 @@ size_t layout_small_smem(const LayoutArgs &a);
 size_t layout_pos_smem(const LayoutArgs &a);
 cudaError_t launch_dispatch(const DispatchArgs &a, bool fp8, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
 
 // Per-device facts, cached.
 struct DeviceInfo {

@@ -34,7 +34,7 @@ EP_ERR_SCRATCH_LIMIT = 8
 ABI_SYMBOLS = (
     "ep_status_str", "ep_max_recv_rows", "ep_layout", "ep_dispatch", "ep_combine",
     "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
-    "ep_handle_check", "ep_layout_noalloc",
+    "ep_handle_check", "ep_layout_noalloc", "ep_dispatch_backward", "ep_combine_backward",
 )
 
 
@@ -85,6 +85,10 @@ def lib() -> ctypes.CDLL:
         L.ep_handle_check.restype = I
         L.ep_layout_noalloc.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
         L.ep_layout_noalloc.restype = I
+        L.ep_dispatch_backward.argtypes = [P, P, I, S, P, P]
+        L.ep_dispatch_backward.restype = I
+        L.ep_combine_backward.argtypes = [P, P, P, P, I, S, P, P, P]
+        L.ep_combine_backward.restype = I
         _LIB = L
     return _LIB
 
@@ -249,6 +253,43 @@ def ep_combine(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,
                           _stream(stream))
     _check(st, "ep_combine")
     return out
+
+
+def ep_dispatch_backward(handle: Handle, grad_recv: torch.Tensor, grad_x: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """grad_x [T, H] bf16 = sum of each token's receive-row gradients."""
+    rows, H = grad_recv.shape
+    if grad_x is None:
+        grad_x = torch.empty(handle.num_tokens, H, dtype=torch.bfloat16, device=grad_recv.device)
+    st = lib().ep_dispatch_backward(handle.ptr, _dev_ptr(grad_recv, torch.bfloat16, "grad_recv"), H, rows,
+                                    _dev_ptr(grad_x, torch.bfloat16, "grad_x", (handle.num_tokens, H)),
+                                    _stream(stream))
+    _check(st, "ep_dispatch_backward")
+    return grad_x
+
+
+def ep_combine_backward(handle: Handle, grad_out: torch.Tensor, topk_weights: torch.Tensor,
+                        y: Optional[torch.Tensor] = None, grad_y: Optional[torch.Tensor] = None,
+                        grad_weights: Optional[torch.Tensor] = None, want_grad_weights: bool = True,
+                        stream=None):
+    """Returns (grad_y [rows, H] bf16, grad_weights [T, k] fp32 or None)."""
+    T, H = grad_out.shape
+    rows = handle.num_recv_rows if y is None else y.shape[0]
+    if grad_y is None:
+        grad_y = torch.empty(rows, H, dtype=torch.bfloat16, device=grad_out.device)
+    if want_grad_weights and grad_weights is None:
+        grad_weights = torch.empty(T, handle.num_topk, dtype=torch.float32, device=grad_out.device)
+    if not want_grad_weights:
+        grad_weights = None
+    st = lib().ep_combine_backward(handle.ptr, _dev_ptr(grad_out, torch.bfloat16, "grad_out", (handle.num_tokens, H)),
+                                   _dev_ptr(y, torch.bfloat16, "y"),
+                                   _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                            (handle.num_tokens, handle.num_topk)),
+                                   H, grad_y.shape[0], _dev_ptr(grad_y, torch.bfloat16, "grad_y"),
+                                   _dev_ptr(grad_weights, torch.float32, "grad_weights",
+                                            (handle.num_tokens, handle.num_topk)), _stream(stream))
+    _check(st, "ep_combine_backward")
+    return grad_y, grad_weights
 
 
 def ep_handle_free(handle: Handle) -> None:

@@ -147,6 +147,37 @@ ep_status ep_dispatch(const ep_handle *handle, const void *x, int hidden, int us
 ep_status ep_combine(const ep_handle *handle, const void *y, const float *topk_weights,
                      int hidden, size_t recv_rows, void *combined_x, ep_stream_t stream);
 
+/* Dispatch backward.  The pages ("DeepEP (DeepEveryParallel) Documentation",
+ * item 10; news.hada.io "Patrones de uso ...") carry out dispatch's backward
+ * pass with a combine; here it is the combine definition with every weight 1:
+ *   grad_x[t][i] = bf16_rn( fp32 chain over valid slots j in slot order of
+ *                           acc = acc + grad_recv[pos[t][j]][i], from +0.0f )
+ *   grad_recv: device bf16 [recv_rows, H] (gradients of the receive rows; for
+ *     an FP8 dispatch the gradient passes the quantisation unchanged).
+ *   grad_x: device bf16 [T, H].  A token with no valid slot gets +0.0.
+ * No allocation, no host synchronisation. */
+ep_status ep_dispatch_backward(const ep_handle *handle, const void *grad_recv, int hidden,
+                               size_t recv_rows, void *grad_x, ep_stream_t stream);
+
+/* Combine backward (combine's backward pass is a dispatch, same passages):
+ * with g = grad_out[t],
+ *   grad_y[pos[t][j]][i] = bf16_rn( fp32_rn( topk_weights[t][j] * g[i] ) )   (weighted dispatch)
+ *   grad_weights[t][j]   = sum_i g[i] * y[pos[t][j]][i]  accumulated in fp32 (dot product)
+ *   grad_out: device bf16 [T, H]; y: device bf16 [recv_rows, H] (the expert
+ *     outputs combine read; may be NULL when grad_weights is NULL);
+ *   topk_weights: device fp32 [T, k]; grad_y: device bf16 [recv_rows, H]
+ *     (only rows that slots map to are written);
+ *   grad_weights: device fp32 [T, k] or NULL; 0 for unused slots.
+ * grad_y is exact to the stated roundings.  grad_weights is summed in a fixed
+ * order (deterministic run to run): per-thread chains over ceil(H/2048)
+ * groups of 16 products, an xor shuffle tree and a sum over the block's 4
+ * warps, so its error from the exact dot product is at most about
+ * (16*ceil(H/2048) + 37) * 2^-24 * sum_i |g[i]*y[i]|.
+ * No allocation, no host synchronisation. */
+ep_status ep_combine_backward(const ep_handle *handle, const void *grad_out, const void *y,
+                              const float *topk_weights, int hidden, size_t recv_rows,
+                              void *grad_y, float *grad_weights, ep_stream_t stream);
+
 /* Release a handle.  Its device memory is freed stream-ordered on the stream
  * that created it (cudaFreeAsync); work that uses the handle on other streams
  * must be ordered before that stream's current position by the caller.
