@@ -69,6 +69,8 @@ def lib():
         L.oracle_combine.restype = i32
         L.oracle_combine_backward.argtypes = [P, P, i64, i32, P, P, i32, i32, P, P]
         L.oracle_combine_backward.restype = i32
+        L.oracle_dispatch_fp8_prequant.argtypes = [P, P, i32, i32, i32, P, P, P, i64]
+        L.oracle_dispatch_fp8_prequant.restype = i32
         _LIB = L
     return _LIB
 
@@ -198,6 +200,31 @@ def dispatch_fp8(x, pos: np.ndarray, n_rows: int):
     st = lib().oracle_dispatch_fp8(_ptr(xb), T, H, k, _ptr(pos), _ptr(recv), _ptr(scales), n_rows)
     if st != OR_OK:
         raise OracleError(st, "oracle_dispatch_fp8")
+    return recv, scales
+
+
+def quantize_rows(x) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token FP8 quantisation (the dispatch's per-group step) of a whole
+    bf16 [T, H] batch: (codes uint8 [T, H], scales float32 [T, H/128])."""
+    xb = _u16(x)
+    T, H = xb.shape
+    pos = np.arange(T, dtype=np.int32)[:, None]
+    return dispatch_fp8(xb, pos, T)
+
+
+def dispatch_fp8_prequant(xq: np.ndarray, xs: np.ndarray, pos: np.ndarray, n_rows: int):
+    """Dispatch of already-quantised input: bit copies of codes and scales."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    xs = np.ascontiguousarray(xs, dtype=np.float32)
+    T, H = xq.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    k = pos.shape[1]
+    recv = np.zeros((n_rows, H), np.uint8)
+    scales = np.zeros((n_rows, H // 128), np.float32)
+    st = lib().oracle_dispatch_fp8_prequant(_ptr(xq), _ptr(xs), T, H, k, _ptr(pos), _ptr(recv),
+                                            _ptr(scales), n_rows)
+    if st != OR_OK:
+        raise OracleError(st, "oracle_dispatch_fp8_prequant")
     return recv, scales
 
 

@@ -470,3 +470,29 @@ int oracle_combine_backward(const uint16_t *grad_out, const uint16_t *y, int64_t
     }
     return OR_OK;
 }
+
+/* Dispatch of input that is already FP8 ("DeepEP (DeepEveryParallel)
+ * Documentation", item 10: dispatch takes BF16 input, or FP8 input given as
+ * data plus scale factors).  Nothing is requantised: receive row pos[t][j]
+ * becomes a bit copy of the codes xq[t] and of the H/128 scales xs[t]. */
+int oracle_dispatch_fp8_prequant(const uint8_t *xq, const float *xs, int T, int H, int k,
+                                 const int32_t *pos, uint8_t *recv, float *scales, int64_t n_rows) {
+    if (T < 0 || H < 128 || H % 128 != 0 || k < 1) {
+        return OR_ERR_INVALID_ARG;
+    }
+    int G = H / 128;
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int32_t p = pos[(int64_t)t * k + j];
+            if (p < 0) {
+                continue;
+            }
+            if (p >= n_rows) {
+                return OR_ERR_INVALID_ARG;
+            }
+            memcpy(recv + (int64_t)p * H, xq + (int64_t)t * H, (size_t)H);
+            memcpy(scales + (int64_t)p * G, xs + (int64_t)t * G, (size_t)G * sizeof(float));
+        }
+    }
+    return OR_OK;
+}

@@ -248,3 +248,21 @@ def test_combine_is_fused(orc):
     w = np.array([[1.0 + 2.0 ** -20, 1.0 + 2.0 ** -20]], np.float32)
     out = orc.combine(y, w, np.array([[0, 1]], np.int32))
     assert orc.bf16_to_f32(int(out[0, 0])) == -(2.0 ** -27)
+
+
+# --- pre-quantised FP8 input -------------------------------------------------
+
+@pytest.mark.parametrize("name", ["prefill", "decode"])
+def test_prequant_dispatch_equals_quantise_then_dispatch(orc, name):
+    """Quantising each token first and dispatching the codes gives exactly the
+    fused FP8 dispatch; and every received row is its source token's row."""
+    w = W.WORKLOADS[name].scaled(T=64)
+    x, idx, _ = W.make_routing(w)
+    _, L = orc.layout(idx.numpy(), w.E, w.R, capacity=w.capacity)
+    xq, xs = orc.quantize_rows(x)
+    q1, s1 = orc.dispatch_fp8_prequant(xq, xs, L.pos, L.n_rows)
+    q2, s2 = orc.dispatch_fp8(x, L.pos, L.n_rows)
+    assert (q1 == q2).all() and (s1.view(np.uint32) == s2.view(np.uint32)).all()
+    rows = np.nonzero(L.src_idx >= 0)[0]
+    assert (q1[rows] == xq[L.src_idx[rows]]).all()
+    assert (s1[rows] == xs[L.src_idx[rows]]).all()
