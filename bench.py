@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-cpu-baseline] [--no-e2e] [--no-decode]
-                    [--no-backward]
+                    [--no-backward] [--no-overlap]
 
 A step is one pass of the whole path over one batch: ep_layout (2 kernels),
 ep_dispatch (FP8 e4m3 or BF16), ep_combine (BF16), all through the C ABI.
@@ -67,6 +67,7 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-backward", action="store_true")
+    p.add_argument("--no-overlap", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
 
@@ -515,6 +516,10 @@ def run_ours(args, w):
     if not args.no_backward:
         backward = run_backward(w, dev, ep, idx, tw, y, flush_l2)
 
+    overlap = None
+    if not args.no_overlap:
+        overlap = run_overlap(w, dev, ep, idx, x, tw, y, flush_l2)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed)
@@ -527,7 +532,7 @@ def run_ours(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "decode": decode, "backward": backward,
+            "decode": decode, "backward": backward, "overlap": overlap,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "wall_s": wall,
             "host_us_per_step": host_s * 1e6,
         }
@@ -661,6 +666,66 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
     c_bytes = T * H * 2 + V * H * 2 + T * k * 8 + V * H * 2 + T * k * 4
     return {"dispatch_backward": {"us": d_us, "bytes": d_bytes, "gbs": d_bytes / d_us / 1e3},
             "combine_backward": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3}}
+
+
+def run_overlap(w, dev, ep, idx_dev, x_dev, tw_dev, y_dev, flush_l2, reps: int = 10) -> dict:
+    """SM-budgeted communication overlapped with compute: a bf16 GEMM of the
+    expert-GEMM shape [T, H] x [H, 4096] (cuBLAS, the stand-in for the work
+    the budget leaves SMs to) on the current stream, and dispatch + combine
+    with num_sms = n on a second stream.  Reports each alone and both
+    together (device time from the first launch to the last completion)."""
+    res = ep.ep_layout(idx_dev, w.E, w.R, w.align, w.capacity)
+    h = res.handle
+    rows = h.num_recv_rows
+    rdt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
+    recv = torch.empty(rows, w.H, dtype=rdt, device=dev)
+    sc = torch.empty(rows, w.H // 128, dtype=torch.float32, device=dev) if w.fp8 else None
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    g = torch.Generator(device=dev).manual_seed(3)
+    wt = torch.randn(w.H, 4096, generator=g, device=dev).to(torch.bfloat16)
+    act = torch.randn(w.T, w.H, generator=g, device=dev).to(torch.bfloat16)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side_hi = torch.cuda.Stream(priority=-1)  # high priority: scheduled first as SMs free up
+
+    def comm(n):
+        ep.ep_dispatch_ex(h, x_dev, w.fp8, recv_x=recv, recv_scales=sc, num_sms=n)
+        ep.ep_combine_ex(h, y_dev, tw_dev, out=out, num_sms=n)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush_l2()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(GPU_LEAD_CYCLES // 2)
+            e0.record(main)
+            fn()
+            e1.record(main)
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.mean(ts)
+
+    def gemm():
+        torch.matmul(act, wt)
+
+    def both(n, stream):
+        stream.wait_stream(main)
+        with torch.cuda.stream(stream):
+            comm(n)
+        gemm()
+        main.wait_stream(stream)
+
+    out_d = {"gemm_us": timed(gemm)}
+    for n in (16, 32, 64, 0):
+        key = "all" if n == 0 else str(n)
+        out_d["comm_us_sms_" + key] = timed(lambda: comm(n))
+        out_d["both_us_sms_" + key] = timed(lambda: both(n, side))
+        out_d["both_hiprio_us_sms_" + key] = timed(lambda: both(n, side_hi))
+    h.free()
+    return out_d
 
 
 def run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y_dev, nbytes, world):

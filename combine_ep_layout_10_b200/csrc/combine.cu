@@ -68,20 +68,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
-template <int VPT>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
+template <int VPT, bool LOOP>
+__global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(CombineArgs a) {
     __shared__ int32_t p_s[kMaxTopk];
     __shared__ float w_s[kMaxTopk];
     pdl_wait_then_trigger();
-    const int t = blockIdx.x / a.blocks_per_token;
-    const int cb = blockIdx.x - t * a.blocks_per_token;
+    const size_t row_bytes = (size_t)a.H * 2;
+    const int nblocks = a.T * a.blocks_per_token;  // < 2^31, checked on the host
+    // One (token, vector block) pair per block unless the grid is capped
+    // (LOOP): then a grid stride over the pairs.
+#pragma unroll 1
+    for (int b = blockIdx.x; b < nblocks; b += gridDim.x) {
+    const int t = b / a.blocks_per_token;
+    const int cb = b - t * a.blocks_per_token;
     if (threadIdx.x < a.k) {
         p_s[threadIdx.x] = __ldg(a.pos + (int64_t)t * a.k + threadIdx.x);
         w_s[threadIdx.x] = a.w != nullptr ? __ldg(a.w + (int64_t)t * a.k + threadIdx.x) : 1.0f;
     }
     __syncthreads();
 
-    const size_t row_bytes = (size_t)a.H * 2;
 #pragma unroll
     for (int vi = 0; vi < VPT; ++vi) {
         const int v = (cb * VPT + vi) * kCombineThreads + threadIdx.x;
@@ -109,21 +114,32 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
         o.w = pack_bf16x2(acc[6], acc[7]);
         st_out_v4(a.out + (size_t)t * row_bytes + (size_t)v * 16, o);
     }
+    if (!LOOP) break;
+    __syncthreads();  // p_s / w_s are rewritten for the next pair
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
-    const long long blocks = (long long)a.T * a.blocks_per_token;
+    long long blocks = (long long)a.T * a.blocks_per_token;
     if ((long long)a.blocks_per_token * a.vpt * kCombineThreads < a.nvec)
         return cudaErrorInvalidConfiguration;
-    switch (a.vpt) {
-        case 1: return launch_kernel(combine_kernel<1>, (unsigned)blocks, kCombineThreads, 0, s, a);
-        case 2: return launch_kernel(combine_kernel<2>, (unsigned)blocks, kCombineThreads, 0, s, a);
-        case 4: return launch_kernel(combine_kernel<4>, (unsigned)blocks, kCombineThreads, 0, s, a);
-        default: return cudaErrorInvalidConfiguration;
+    const bool loop = a.num_sms > 0;
+    void (*kernel)(CombineArgs) = nullptr;
+    if (a.vpt == 1) kernel = loop ? combine_kernel<1, true> : combine_kernel<1, false>;
+    if (a.vpt == 2) kernel = loop ? combine_kernel<2, true> : combine_kernel<2, false>;
+    if (a.vpt == 4) kernel = loop ? combine_kernel<4, true> : combine_kernel<4, false>;
+    if (kernel == nullptr) return cudaErrorInvalidConfiguration;
+    if (loop) {
+        int per_sm = 0;
+        cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCombineThreads, 0);
+        if (err != cudaSuccess) return err;
+        const long long cap = (long long)a.num_sms * (per_sm > 0 ? per_sm : 1);
+        if (cap < blocks) blocks = cap;
     }
+    return launch_kernel(kernel, (unsigned)blocks, kCombineThreads, 0, s, a);
 }
 
 }  // namespace ep

@@ -19,6 +19,10 @@
 //     round-to-nearest-even satfinite e4m3 conversion give 16 code bytes; the
 //     group's first lane writes the scale.
 //   * BF16: a thread owns two 16-byte vectors a block apart and copies them.
+//   * FP8 input already quantised (codes + scales): a thread copies 16 codes,
+//     the group's first lane copies the scale.
+// FP8 scales are written at p * s_row + g * s_grp (row-major [rows, H/128],
+// or column-major with a caller-chosen leading dimension for FP8 GEMMs).
 // A TMA variant (bulk load into a shared ring, k bulk stores from shared
 // memory) was measured slower on this path: bulk stores of scattered 7-14 KB
 // rows sustain less write bandwidth on B200 than plain 16-byte stores.
@@ -52,98 +56,162 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     f[7] = bf16_bits_to_f32(v.w >> 16);
 }
 
+// The kernels take one (token, chunk) unit per block; when the caller caps
+// the grid (num_sms) the LOOP instantiation walks the units with a grid stride.
+
+template <bool LOOP>
 __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
     __shared__ int32_t p_s[kMaxTopk];
     pdl_wait_then_trigger();
-    const int t = blockIdx.x / a.nchunks;
-    const int c = blockIdx.x - t * a.nchunks;
-    const int ch0 = c * a.chunk;
-    const int chn = min(a.chunk, a.H - ch0);
     const int tid = threadIdx.x;
-    if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
-    const int ch = ch0 + tid * 16;
-    const bool act = tid * 16 < chn;
-    uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-    if (act) {
-        const uint8_t *src = a.x + ((int64_t)t * a.H + ch) * 2;
-        v0 = ld_nc_v4(src);
-        v1 = ld_nc_v4(src + 16);
-    }
-    __syncthreads();
-    float f[16];
-    unpack8(v0, f);
-    unpack8(v1, f + 8);
-    float amax = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(f[q]));
-    // A 128-channel group is 8 consecutive lanes: xor distances < 8 stay inside it.
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    if (!act) return;
-    uint4 q16 = make_uint4(0u, 0u, 0u, 0u);
-    float scale = 0.0f;
-    if (amax != 0.0f) {
-        scale = __fdiv_rn(amax, 448.0f);
-        const float inv = __fdiv_rn(448.0f, amax);
-        uint32_t b[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float2 pr = make_float2(__fmul_rn(f[2 * q], inv), __fmul_rn(f[2 * q + 1], inv));
-            b[q] = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
-        }
-        q16.x = b[0] | (b[1] << 16);
-        q16.y = b[2] | (b[3] << 16);
-        q16.z = b[4] | (b[5] << 16);
-        q16.w = b[6] | (b[7] << 16);
-    }
-    const int G_row = a.H / 128;
     const bool leader = (tid & 7) == 0;
-    for (int j = 0; j < a.k; ++j) {
-        const int p = p_s[j];
-        if (p < 0) continue;
-        *reinterpret_cast<uint4 *>(a.recv + (int64_t)p * a.H + ch) = q16;
-        if (leader) a.scales[(int64_t)p * G_row + ch / 128] = scale;
+    // One unit per block unless the grid is capped (LOOP): then a grid stride.
+    for (int u = blockIdx.x; u < a.nunits; u += gridDim.x) {
+        const int t = u / a.nchunks;
+        const int ch0 = (u - t * a.nchunks) * a.chunk;
+        const int chn = min(a.chunk, a.H - ch0);
+        if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
+        const int ch = ch0 + tid * 16;
+        const bool act = tid * 16 < chn;
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (act) {
+            const uint8_t *src = a.x + ((int64_t)t * a.H + ch) * 2;
+            v0 = ld_nc_v4(src);
+            v1 = ld_nc_v4(src + 16);
+        }
+        __syncthreads();
+        float f[16];
+        unpack8(v0, f);
+        unpack8(v1, f + 8);
+        float amax = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(f[q]));
+        // A 128-channel group is 8 consecutive lanes: xor distances < 8 stay inside it.
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        if (act) {
+            uint4 q16 = make_uint4(0u, 0u, 0u, 0u);
+            float scale = 0.0f;
+            if (amax != 0.0f) {
+                scale = __fdiv_rn(amax, 448.0f);
+                const float inv = __fdiv_rn(448.0f, amax);
+                uint32_t b[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float2 pr = make_float2(__fmul_rn(f[2 * q], inv), __fmul_rn(f[2 * q + 1], inv));
+                    b[q] = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
+                }
+                q16.x = b[0] | (b[1] << 16);
+                q16.y = b[2] | (b[3] << 16);
+                q16.z = b[4] | (b[5] << 16);
+                q16.w = b[6] | (b[7] << 16);
+            }
+            const int g = ch / 128;
+            for (int j = 0; j < a.k; ++j) {
+                const int p = p_s[j];
+                if (p < 0) continue;
+                *reinterpret_cast<uint4 *>(a.recv + (int64_t)p * a.H + ch) = q16;
+                if (leader) a.scales[(int64_t)p * a.s_row + (int64_t)g * a.s_grp] = scale;
+            }
+        }
+        if (!LOOP) break;
+        __syncthreads();  // p_s is rewritten by the next unit
     }
 }
 
+// Pre-quantised FP8 input: codes and scales are copied, not recomputed.
+template <bool LOOP>
+__global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) {
+    __shared__ int32_t p_s[kMaxTopk];
+    pdl_wait_then_trigger();
+    const int tid = threadIdx.x;
+    const bool leader = (tid & 7) == 0;
+    const int G_row = a.H / 128;
+    // One unit per block unless the grid is capped (LOOP): then a grid stride.
+    for (int u = blockIdx.x; u < a.nunits; u += gridDim.x) {
+        const int t = u / a.nchunks;
+        const int ch0 = (u - t * a.nchunks) * a.chunk;
+        const int chn = min(a.chunk, a.H - ch0);
+        if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
+        const int ch = ch0 + tid * 16;
+        const bool act = tid * 16 < chn;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        float scale = 0.0f;
+        if (act) {
+            v = ld_nc_v4(a.x + (int64_t)t * a.H + ch);
+            if (leader) scale = __ldg(a.x_scales + (int64_t)t * G_row + ch / 128);
+        }
+        __syncthreads();
+        if (act) {
+            const int g = ch / 128;
+            for (int j = 0; j < a.k; ++j) {
+                const int p = p_s[j];
+                if (p < 0) continue;
+                *reinterpret_cast<uint4 *>(a.recv + (int64_t)p * a.H + ch) = v;
+                if (leader) a.scales[(int64_t)p * a.s_row + (int64_t)g * a.s_grp] = scale;
+            }
+        }
+        if (!LOOP) break;
+        __syncthreads();  // p_s is rewritten by the next unit
+    }
+}
+
+template <bool LOOP>
 __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchArgs a) {
     __shared__ int32_t p_s[kMaxTopk];
     pdl_wait_then_trigger();
-    const int t = blockIdx.x / a.nchunks;
-    const int c = blockIdx.x - t * a.nchunks;
-    const int ch0 = c * a.chunk;
-    const int chn = min(a.chunk, a.H - ch0);
     const int tid = threadIdx.x;
-    if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
-    // Two 16-byte vectors per thread, a block apart, so that every warp-wide
-    // load and store covers 512 contiguous bytes.
-    const int nv = chn / 8;
-    const int u0 = tid, u1 = tid + blockDim.x;
-    const bool act0 = u0 < nv, act1 = u1 < nv;
-    uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-    const uint8_t *src = a.x + ((int64_t)t * a.H + ch0) * 2;
-    if (act0) v0 = ld_nc_v4(src + (size_t)u0 * 16);
-    if (act1) v1 = ld_nc_v4(src + (size_t)u1 * 16);
-    __syncthreads();
-    if (!act0) return;
-    for (int j = 0; j < a.k; ++j) {
-        const int p = p_s[j];
-        if (p < 0) continue;
-        uint8_t *dst = a.recv + ((int64_t)p * a.H + ch0) * 2;
-        *reinterpret_cast<uint4 *>(dst + (size_t)u0 * 16) = v0;
-        if (act1) *reinterpret_cast<uint4 *>(dst + (size_t)u1 * 16) = v1;
+    // One unit per block unless the grid is capped (LOOP): then a grid stride.
+    for (int u = blockIdx.x; u < a.nunits; u += gridDim.x) {
+        const int t = u / a.nchunks;
+        const int ch0 = (u - t * a.nchunks) * a.chunk;
+        const int chn = min(a.chunk, a.H - ch0);
+        if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
+        // Two 16-byte vectors per thread, a block apart, so that every warp-wide
+        // load and store covers 512 contiguous bytes.
+        const int nv = chn / 8;
+        const int u0 = tid, u1 = tid + blockDim.x;
+        const bool act0 = u0 < nv, act1 = u1 < nv;
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        const uint8_t *src = a.x + ((int64_t)t * a.H + ch0) * 2;
+        if (act0) v0 = ld_nc_v4(src + (size_t)u0 * 16);
+        if (act1) v1 = ld_nc_v4(src + (size_t)u1 * 16);
+        __syncthreads();
+        if (act0) {
+            for (int j = 0; j < a.k; ++j) {
+                const int p = p_s[j];
+                if (p < 0) continue;
+                uint8_t *dst = a.recv + ((int64_t)p * a.H + ch0) * 2;
+                *reinterpret_cast<uint4 *>(dst + (size_t)u0 * 16) = v0;
+                if (act1) *reinterpret_cast<uint4 *>(dst + (size_t)u1 * 16) = v1;
+            }
+        }
+        if (!LOOP) break;
+        __syncthreads();  // p_s is rewritten by the next unit
     }
 }
 
 }  // namespace
 
-cudaError_t launch_dispatch(const DispatchArgs &a, bool fp8, cudaStream_t st) {
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
     if (a.nunits == 0) return cudaSuccess;
     // One block per unit, one thread per 16 channels (chunk <= 8192 -> <= 512 threads).
     const int threads = (((a.chunk + 15) / 16 + 31) / 32) * 32;
-    return launch_kernel(fp8 ? dispatch_fp8_kernel : dispatch_bf16_kernel, (unsigned)a.nunits, threads, 0, st,
-                         a);
+    const bool loop = a.num_sms > 0;
+    void (*kernel)(DispatchArgs) =
+        a.mode == kDispatchQuantFp8 ? (loop ? dispatch_fp8_kernel<true> : dispatch_fp8_kernel<false>)
+        : a.mode == kDispatchCopyFp8 ? (loop ? dispatch_fp8_copy_kernel<true> : dispatch_fp8_copy_kernel<false>)
+                                     : (loop ? dispatch_bf16_kernel<true> : dispatch_bf16_kernel<false>);
+    int grid = a.nunits;
+    if (loop) {
+        int per_sm = 0;
+        cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
+        if (err != cudaSuccess) return err;
+        const long long cap = (long long)a.num_sms * (per_sm > 0 ? per_sm : 1);
+        if (cap < grid) grid = (int)cap;
+    }
+    return launch_kernel(kernel, (unsigned)grid, threads, 0, st, a);
 }
 
 }  // namespace ep

@@ -216,16 +216,30 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     return EP_OK;
 }
 
-ep_status ep_dispatch(const ep_handle *h, const void *x, int H, int use_fp8, void *recv_x,
-                      float *recv_scales, int32_t *recv_src_idx, size_t recv_rows,
-                      ep_stream_t stream) {
-    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
-    if (use_fp8 && H % 128 != 0) return EP_ERR_INVALID_ARG;
+ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scales, int H, int in_format,
+                         int out_format, void *recv_x, float *recv_scales, int64_t scale_row_stride,
+                         int64_t scale_group_stride, int32_t *recv_src_idx, size_t recv_rows, int num_sms,
+                         ep_stream_t stream) {
+    if (h == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
+    const bool in_fp8 = in_format == EP_FORMAT_E4M3;
+    const bool out_fp8 = out_format == EP_FORMAT_E4M3;
+    if ((in_format != EP_FORMAT_BF16 && !in_fp8) || (out_format != EP_FORMAT_BF16 && !out_fp8))
+        return EP_ERR_INVALID_ARG;
+    if (in_fp8 && !out_fp8) return EP_ERR_INVALID_ARG;  // no dequantising dispatch
+    if (out_fp8 && H % 128 != 0) return EP_ERR_INVALID_ARG;
     if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    const int64_t G = H / 128;
+    if (out_fp8) {
+        // Non-overlapping scale layouts only: row-major-like or column-major-like.
+        const bool row_like = scale_group_stride == 1 && scale_row_stride >= G;
+        const bool col_like = scale_row_stride == 1 && scale_group_stride >= (int64_t)recv_rows;
+        if (!(row_like || col_like)) return EP_ERR_INVALID_ARG;
+    }
     if (h->T > 0) {
         if (x == nullptr || recv_x == nullptr || !aligned(x, 16) || !aligned(recv_x, 16))
             return EP_ERR_INVALID_ARG;
-        if (use_fp8 && (recv_scales == nullptr || !aligned(recv_scales, 4))) return EP_ERR_INVALID_ARG;
+        if (out_fp8 && (recv_scales == nullptr || !aligned(recv_scales, 4))) return EP_ERR_INVALID_ARG;
+        if (in_fp8 && (x_scales == nullptr || !aligned(x_scales, 4))) return EP_ERR_INVALID_ARG;
     }
     if (recv_src_idx != nullptr && !aligned(recv_src_idx, 4)) return EP_ERR_INVALID_ARG;
     int dev;
@@ -234,28 +248,40 @@ ep_status ep_dispatch(const ep_handle *h, const void *x, int H, int use_fp8, voi
     if (st != EP_OK) return st;
     if (dev != h->device) return EP_ERR_INVALID_ARG;
 
-    const int align_ch = use_fp8 ? 128 : 8;
+    const int align_ch = out_fp8 ? 128 : 8;
     const int nchunks = (H + kMaxChunkChannels - 1) / kMaxChunkChannels;
     const int chunk = (int)round_up((size_t)((H + nchunks - 1) / nchunks), align_ch);
 
     DispatchArgs a{};
     a.x = static_cast<const uint8_t *>(x);
+    a.x_scales = x_scales;
     a.pos = h->pos;
     a.recv = static_cast<uint8_t *>(recv_x);
     a.scales = recv_scales;
+    a.s_row = scale_row_stride;
+    a.s_grp = scale_group_stride;
+    a.mode = !out_fp8 ? kDispatchCopyBf16 : in_fp8 ? kDispatchCopyFp8 : kDispatchQuantFp8;
+    a.num_sms = num_sms;
     a.T = h->T; a.k = h->k; a.H = H;
     a.chunk = chunk;
     a.nchunks = (H + chunk - 1) / chunk;
-    a.nunits = (long long)h->T * a.nchunks;
-    cudaError_t e = launch_dispatch(a, use_fp8 != 0, stream);
+    if ((int64_t)h->T * a.nchunks >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
+    a.nunits = h->T * a.nchunks;
+    cudaError_t e = launch_dispatch(a, stream);
     if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)
         e = cudaMemcpyAsync(recv_src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
     return cuda_status(e);
 }
 
-ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int H, size_t recv_rows,
-                     void *out, ep_stream_t stream) {
-    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+ep_status ep_dispatch(const ep_handle *h, const void *x, int H, int use_fp8, void *recv_x,
+                      float *recv_scales, int32_t *recv_src_idx, size_t recv_rows, ep_stream_t stream) {
+    return ep_dispatch_ex(h, x, nullptr, H, EP_FORMAT_BF16, use_fp8 ? EP_FORMAT_E4M3 : EP_FORMAT_BF16, recv_x,
+                          recv_scales, H / 128, 1, recv_src_idx, recv_rows, 0, stream);
+}
+
+ep_status ep_combine_ex(const ep_handle *h, const void *y, const float *topk_w, int H, size_t recv_rows,
+                        void *out, int num_sms, ep_stream_t stream) {
+    if (h == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
     if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
     if (h->T > 0) {
         if (y == nullptr || out == nullptr || topk_w == nullptr) return EP_ERR_INVALID_ARG;
@@ -276,7 +302,14 @@ ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int
     a.nvec = H / 8;
     a.vpt = EP_COMBINE_VPT;
     a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
+    if ((int64_t)h->T * a.blocks_per_token >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
+    a.num_sms = num_sms;
     return cuda_status(launch_combine(a, stream));
+}
+
+ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int H, size_t recv_rows,
+                     void *out, ep_stream_t stream) {
+    return ep_combine_ex(h, y, topk_w, H, recv_rows, out, 0, stream);
 }
 
 ep_status ep_dispatch_backward(const ep_handle *h, const void *grad_recv, int H, size_t recv_rows,
@@ -299,6 +332,8 @@ ep_status ep_dispatch_backward(const ep_handle *h, const void *grad_recv, int H,
     a.nvec = H / 8;
     a.vpt = EP_COMBINE_VPT;
     a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
+    if ((int64_t)h->T * a.blocks_per_token >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
+    a.num_sms = 0;
     return cuda_status(launch_combine(a, stream));
 }
 

@@ -157,15 +157,23 @@ struct LayoutArgs {
     uint8_t *out_in_rank;
 };
 
+constexpr int kDispatchCopyBf16 = 0;  // bf16 in, bf16 rows out
+constexpr int kDispatchQuantFp8 = 1;  // bf16 in, e4m3 rows + scales out (quantised here)
+constexpr int kDispatchCopyFp8 = 2;   // e4m3 + scales in (already quantised), copied out
+
 struct DispatchArgs {
-    const uint8_t *x;        // bf16 [T, H]
+    const uint8_t *x;        // bf16 [T, H], or e4m3 [T, H] for kDispatchCopyFp8
+    const float *x_scales;   // [T, H/128] row-major, kDispatchCopyFp8 only
     const int32_t *pos;      // [T, k]
     uint8_t *recv;           // [rows, H] bf16 or e4m3
-    float *scales;           // [rows, H/128] (FP8 only)
+    float *scales;           // element (p, g) at p * s_row + g * s_grp (FP8 only)
+    int64_t s_row, s_grp;
+    int mode;                // kDispatch*
+    int num_sms;             // 0: one block per unit; else grid capped to num_sms SMs' worth
     int T, k, H;
-    int chunk;               // channels per work unit (block)
+    int chunk;               // channels per work unit
     int nchunks;             // units per token
-    long long nunits;        // T * nchunks
+    int nunits;              // T * nchunks (< 2^31, checked on the host)
 };
 
 struct CombineArgs {
@@ -177,6 +185,7 @@ struct CombineArgs {
     int nvec;                // H / 8 (16-byte vectors per row)
     int vpt;                 // vectors per thread: 1, 2 or 4
     int blocks_per_token;    // ceil(nvec / (128 * vpt))
+    int num_sms;             // 0: one block per (token, vector block); else grid capped
 };
 
 struct CombineBwdArgs {
@@ -194,7 +203,7 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 size_t layout_count_smem(const LayoutArgs &a);
 size_t layout_small_smem(const LayoutArgs &a);
 size_t layout_pos_smem(const LayoutArgs &a);
-cudaError_t launch_dispatch(const DispatchArgs &a, bool fp8, cudaStream_t s);
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
 

@@ -35,7 +35,11 @@ ABI_SYMBOLS = (
     "ep_status_str", "ep_max_recv_rows", "ep_layout", "ep_dispatch", "ep_combine",
     "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
     "ep_handle_check", "ep_layout_noalloc", "ep_dispatch_backward", "ep_combine_backward",
+    "ep_dispatch_ex", "ep_combine_ex",
 )
+
+EP_FORMAT_BF16 = 0
+EP_FORMAT_E4M3 = 1
 
 
 class EpError(RuntimeError):
@@ -89,6 +93,11 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_backward.restype = I
         L.ep_combine_backward.argtypes = [P, P, P, P, I, S, P, P, P]
         L.ep_combine_backward.restype = I
+        I64 = ctypes.c_int64
+        L.ep_dispatch_ex.argtypes = [P, P, P, I, I, I, P, P, I64, I64, P, S, I, P]
+        L.ep_dispatch_ex.restype = I
+        L.ep_combine_ex.argtypes = [P, P, P, I, S, P, I, P]
+        L.ep_combine_ex.restype = I
         _LIB = L
     return _LIB
 
@@ -252,6 +261,62 @@ def ep_combine(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,
                           H, rows, _dev_ptr(out, torch.bfloat16, "out", (handle.num_tokens, H)),
                           _stream(stream))
     _check(st, "ep_combine")
+    return out
+
+
+def ep_dispatch_ex(handle: Handle, x: torch.Tensor, out_fp8: bool, x_scales: Optional[torch.Tensor] = None,
+                   recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
+                   scale_layout: str = "row", scale_ld: Optional[int] = None,
+                   recv_src_idx: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None):
+    """Dispatch with input format (bf16, or e4m3 codes + x_scales), scale
+    layout ("row": [rows, H/128]; "col": [H/128, scale_ld]) and SM budget.
+    Returns (recv_x, recv_scales or None, recv_src_idx or None)."""
+    T, H = x.shape
+    if T != handle.num_tokens:
+        raise ValueError("x has %d tokens, the handle %d" % (T, handle.num_tokens))
+    in_fp8 = x.dtype == torch.float8_e4m3fn
+    if in_fp8 and not out_fp8:
+        raise ValueError("e4m3 input needs e4m3 output")
+    rows = handle.num_recv_rows if recv_x is None else recv_x.shape[0]
+    dt = torch.float8_e4m3fn if out_fp8 else torch.bfloat16
+    if recv_x is None:
+        recv_x = torch.empty(rows, H, dtype=dt, device=x.device)
+    G = H // 128
+    s_row, s_grp = G, 1
+    if out_fp8:
+        if scale_layout == "col":
+            ld = scale_ld if scale_ld is not None else (rows + 3) // 4 * 4
+            s_row, s_grp = 1, ld
+            if recv_scales is None:
+                recv_scales = torch.empty(G, ld, dtype=torch.float32, device=x.device)
+        elif scale_layout == "row":
+            if recv_scales is None:
+                recv_scales = torch.empty(rows, G, dtype=torch.float32, device=x.device)
+        else:
+            raise ValueError("scale_layout must be 'row' or 'col'")
+    st = lib().ep_dispatch_ex(handle.ptr, _dev_ptr(x, None, "x"),
+                              _dev_ptr(x_scales, torch.float32, "x_scales", (T, G)) if in_fp8 else None,
+                              H, EP_FORMAT_E4M3 if in_fp8 else EP_FORMAT_BF16,
+                              EP_FORMAT_E4M3 if out_fp8 else EP_FORMAT_BF16,
+                              _dev_ptr(recv_x, dt, "recv_x"),
+                              _dev_ptr(recv_scales, torch.float32, "recv_scales") if out_fp8 else None,
+                              s_row, s_grp, _dev_ptr(recv_src_idx, torch.int32, "recv_src_idx"),
+                              rows, num_sms, _stream(stream))
+    _check(st, "ep_dispatch_ex")
+    return recv_x, (recv_scales if out_fp8 else None), recv_src_idx
+
+
+def ep_combine_ex(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,
+                  out: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None) -> torch.Tensor:
+    rows, H = y.shape
+    if out is None:
+        out = torch.empty(handle.num_tokens, H, dtype=torch.bfloat16, device=y.device)
+    st = lib().ep_combine_ex(handle.ptr, _dev_ptr(y, torch.bfloat16, "y"),
+                             _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                      (handle.num_tokens, handle.num_topk)),
+                             H, rows, _dev_ptr(out, torch.bfloat16, "out", (handle.num_tokens, H)),
+                             num_sms, _stream(stream))
+    _check(st, "ep_combine_ex")
     return out
 
 

@@ -178,6 +178,44 @@ ep_status ep_combine_backward(const ep_handle *handle, const void *grad_out, con
                               const float *topk_weights, int hidden, size_t recv_rows,
                               void *grad_y, float *grad_weights, ep_stream_t stream);
 
+/* Element formats of ep_dispatch_ex. */
+#define EP_FORMAT_BF16 0
+#define EP_FORMAT_E4M3 1
+
+/* Dispatch with the options of the pages' full dispatch call ("DeepEP
+ * (DeepEveryParallel) Documentation", item 10: BF16 or FP8 input, the FP8
+ * input given as data plus scale factors; the SM count the call may use, as
+ * "DeepSeek publica DeepEP ..." (news.hada.io), "Interfaz centrada en
+ * ElasticBuffer", lets num_sms be set per call) and a scale layout a grouped
+ * FP8 GEMM can consume ([hada] "Cambios clave de la versión V2": a GEMM
+ * layout).
+ *   in_format / out_format: EP_FORMAT_BF16 -> BF16 (bit copy, as ep_dispatch),
+ *     EP_FORMAT_BF16 -> EP_FORMAT_E4M3 (quantised here, as ep_dispatch), or
+ *     EP_FORMAT_E4M3 -> EP_FORMAT_E4M3: x is device e4m3 [T, H] already
+ *     quantised and x_scales device fp32 [T, H/128] row-major; codes and
+ *     scales are copied to the k rows unchanged.
+ *   recv_scales: scale of receive row p and group g stored at
+ *     recv_scales[p * scale_row_stride + g * scale_group_stride].  Accepted
+ *     layouts: row-major (group stride 1, row stride >= H/128; ep_dispatch
+ *     uses H/128) and column-major (row stride 1, group stride >= recv_rows,
+ *     e.g. recv_rows rounded up to a multiple of 4 for 16-byte aligned
+ *     columns).  The buffer must hold (recv_rows-1)*row_stride +
+ *     (H/128-1)*group_stride + 1 floats.
+ *   num_sms: 0 = no limit (one block per token chunk); n > 0 = at most the
+ *     blocks n SMs can hold at once, looping over the work, so that
+ *     concurrent kernels on other streams keep the remaining SMs' worth of
+ *     resources (the hardware still places the blocks).
+ * Other arguments and rules as ep_dispatch. */
+ep_status ep_dispatch_ex(const ep_handle *handle, const void *x, const float *x_scales, int hidden,
+                         int in_format, int out_format, void *recv_x, float *recv_scales,
+                         int64_t scale_row_stride, int64_t scale_group_stride,
+                         int32_t *recv_src_idx, size_t recv_rows, int num_sms, ep_stream_t stream);
+
+/* Combine with an SM budget: as ep_combine, with num_sms as in ep_dispatch_ex. */
+ep_status ep_combine_ex(const ep_handle *handle, const void *y, const float *topk_weights,
+                        int hidden, size_t recv_rows, void *combined_x, int num_sms,
+                        ep_stream_t stream);
+
 /* Release a handle.  Its device memory is freed stream-ordered on the stream
  * that created it (cudaFreeAsync); work that uses the handle on other streams
  * must be ordered before that stream's current position by the caller.

@@ -1,0 +1,133 @@
+"""ep_dispatch_ex / ep_combine_ex options against the oracle (GPU).
+
+* pre-quantised FP8 input (codes + scales) is copied bit-exactly;
+* a column-major scale layout holds exactly the row-major scales, transposed;
+* an SM budget (num_sms) changes the launch shape, never the result.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_ep_layout_10_b200 import ep
+from combine_ep_layout_10_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from combine_ep_layout_10_b200 import build
+    build.build()
+    ep.lib()
+    oracle.lib()
+
+
+def u8(t):
+    return t.contiguous().view(torch.uint8).cpu().numpy()
+
+
+def u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def setup(name, T=None):
+    w = W.WORKLOADS[name]
+    w = w.scaled(T=T) if T else w
+    x, idx, tw = W.make_routing(w)
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R, w.align, w.capacity)
+    _, L = oracle.layout(idx.numpy(), w.E, w.R, w.align, w.capacity)
+    return w, x, tw, res, L
+
+
+@pytest.mark.parametrize("name,T", [("prefill", 300), ("decode", None), ("group_limited", 512)])
+def test_prequantised_input(name, T):
+    w, x, tw, res, L = setup(name, T)
+    xq, xs = oracle.quantize_rows(x)
+    xq_d = torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn)
+    xs_d = torch.from_numpy(xs).to(DEV)
+    recv, sc, _ = ep.ep_dispatch_ex(res.handle, xq_d, True, x_scales=xs_d)
+    torch.cuda.synchronize()
+    q, s = oracle.dispatch_fp8_prequant(xq, xs, L.pos, L.n_rows)
+    valid = L.src_idx >= 0
+    assert (u8(recv)[valid] == q[valid]).all()
+    assert (sc.cpu().numpy()[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
+    # and it is the fused FP8 dispatch, exactly
+    q2, s2 = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+    assert (q[valid] == q2[valid]).all() and (s[valid] == s2[valid]).all()
+
+
+@pytest.mark.parametrize("prequant", [False, True])
+def test_column_major_scales(prequant):
+    w, x, tw, res, L = setup("prefill", 257)
+    rows = res.handle.num_recv_rows
+    ld = (rows + 3) // 4 * 4
+    if prequant:
+        xq, xs = oracle.quantize_rows(x)
+        xin = torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn)
+        xsd = torch.from_numpy(xs).to(DEV)
+    else:
+        xin, xsd = x.to(DEV), None
+    sc_col = torch.full((w.H // 128, ld), -3.0, dtype=torch.float32, device=DEV)
+    recv, sc, _ = ep.ep_dispatch_ex(res.handle, xin, True, x_scales=xsd, recv_scales=sc_col,
+                                    scale_layout="col", scale_ld=ld)
+    torch.cuda.synchronize()
+    q, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+    valid = L.src_idx >= 0
+    got = sc.cpu().numpy()
+    assert (got[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
+    assert (got[:, :rows].T[~valid] == -3.0).all() and (got[:, rows:] == -3.0).all()
+    assert (u8(recv)[valid] == q[valid]).all()
+
+
+@pytest.mark.parametrize("num_sms", [1, 3, 16, 1000])
+def test_sm_budget_changes_nothing(num_sms):
+    for name, fp8 in (("group_limited", True), ("large_skewed", False)):
+        w, x, tw, res, L = setup(name, 1024)
+        h = res.handle
+        xd = x.to(DEV)
+        r0, s0, _ = ep.ep_dispatch_ex(h, xd, fp8)
+        r1, s1, _ = ep.ep_dispatch_ex(h, xd, fp8, num_sms=num_sms)
+        y = W.make_expert_out(h.num_recv_rows, w.H, seed=5).to(DEV)
+        twd = tw.to(DEV)
+        o0 = ep.ep_combine_ex(h, y, twd)
+        o1 = ep.ep_combine_ex(h, y, twd, num_sms=num_sms)
+        torch.cuda.synchronize()
+        valid = torch.from_numpy(L.src_idx >= 0).to(DEV)
+        assert torch.equal(r0.view(torch.uint8)[valid], r1.view(torch.uint8)[valid])
+        if fp8:
+            assert torch.equal(s0[valid], s1[valid])
+        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+        assert (u16(o0) == oracle.combine(y.cpu(), tw.numpy(), L.pos)).all()
+
+
+def test_option_errors():
+    w, x, tw, res, L = setup("prefill", 64)
+    h = res.handle
+    xq, xs = oracle.quantize_rows(x)
+    xq_d = torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn)
+    with pytest.raises(ValueError):
+        ep.ep_dispatch_ex(h, xq_d, False, x_scales=torch.from_numpy(xs).to(DEV))
+    L_ = ep.lib()
+    import ctypes
+    rows = h.num_recv_rows
+    recv = torch.empty(rows, w.H, dtype=torch.float8_e4m3fn, device=DEV)
+    sc = torch.empty(rows * (w.H // 128), dtype=torch.float32, device=DEV)
+    P = ctypes.c_void_p
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    G = w.H // 128
+    # overlapping scale strides (row stride smaller than the groups of a row)
+    st = L_.ep_dispatch_ex(h.ptr, P(x.to(DEV).data_ptr()), None, w.H, 0, 1, P(recv.data_ptr()),
+                           P(sc.data_ptr()), G - 1, 1, None, rows, 0, stream)
+    assert st == ep.EP_ERR_INVALID_ARG
+    # e4m3 input without scales
+    st = L_.ep_dispatch_ex(h.ptr, P(xq_d.data_ptr()), None, w.H, 1, 1, P(recv.data_ptr()),
+                           P(sc.data_ptr()), G, 1, None, rows, 0, stream)
+    assert st == ep.EP_ERR_INVALID_ARG
+    # negative SM budget
+    st = L_.ep_dispatch_ex(h.ptr, P(x.to(DEV).data_ptr()), None, w.H, 0, 1, P(recv.data_ptr()),
+                           P(sc.data_ptr()), G, 1, None, rows, -1, stream)
+    assert st == ep.EP_ERR_INVALID_ARG
