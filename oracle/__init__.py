@@ -39,7 +39,13 @@ def lib():
     """Load (building first if needed) the oracle shared library."""
     global _LIB
     if _LIB is None:
-        path = _build.build()
+        _LIB = load(_build.build())
+    return _LIB
+
+
+def load(path: str):
+    """Load an oracle library from `path` and declare its functions."""
+    if True:
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i32, i64 = ctypes.c_int, ctypes.c_int64
@@ -71,8 +77,7 @@ def lib():
         L.oracle_combine_backward.restype = i32
         L.oracle_dispatch_fp8_prequant.argtypes = [P, P, i32, i32, i32, P, P, P, i64]
         L.oracle_dispatch_fp8_prequant.restype = i32
-        _LIB = L
-    return _LIB
+    return L
 
 
 def _ptr(a: np.ndarray):
