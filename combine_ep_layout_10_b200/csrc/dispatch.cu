@@ -45,6 +45,16 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
     return r;
 }
 
+// Store of one 16-byte vector of a receive row.
+__device__ __forceinline__ void st_row_v4(void *p, const uint4 &v) {
+#if EP_DISPATCH_STORE_CS
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+#else
+    *reinterpret_cast<uint4 *>(p) = v;
+#endif
+}
+
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     f[0] = bf16_bits_to_f32(v.x & 0xffffu);
     f[1] = bf16_bits_to_f32(v.x >> 16);
@@ -111,7 +121,7 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
             for (int j = 0; j < a.k; ++j) {
                 const int p = p_s[j];
                 if (p < 0) continue;
-                *reinterpret_cast<uint4 *>(a.recv + (int64_t)p * a.H + ch) = q16;
+                st_row_v4(a.recv + (int64_t)p * a.H + ch, q16);
                 if (leader) a.scales[(int64_t)p * a.s_row + (int64_t)g * a.s_grp] = scale;
             }
         }
@@ -148,7 +158,7 @@ __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) 
             for (int j = 0; j < a.k; ++j) {
                 const int p = p_s[j];
                 if (p < 0) continue;
-                *reinterpret_cast<uint4 *>(a.recv + (int64_t)p * a.H + ch) = v;
+                st_row_v4(a.recv + (int64_t)p * a.H + ch, v);
                 if (leader) a.scales[(int64_t)p * a.s_row + (int64_t)g * a.s_grp] = scale;
             }
         }
@@ -183,8 +193,8 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchArgs a) {
                 const int p = p_s[j];
                 if (p < 0) continue;
                 uint8_t *dst = a.recv + ((int64_t)p * a.H + ch0) * 2;
-                *reinterpret_cast<uint4 *>(dst + (size_t)u0 * 16) = v0;
-                if (act1) *reinterpret_cast<uint4 *>(dst + (size_t)u1 * 16) = v1;
+                st_row_v4(dst + (size_t)u0 * 16, v0);
+                if (act1) st_row_v4(dst + (size_t)u1 * 16, v1);
             }
         }
         if (!LOOP) break;

@@ -14,6 +14,9 @@
 #ifndef EP_DISPATCH_MAX_CHUNK     // dispatch: at most this many channels per work unit
 #define EP_DISPATCH_MAX_CHUNK 8192
 #endif
+#ifndef EP_DISPATCH_STORE_CS      // dispatch: evict-first (.cs) stores of the receive rows
+#define EP_DISPATCH_STORE_CS 0
+#endif
 #ifndef EP_COMBINE_THREADS        // threads per combine block
 #define EP_COMBINE_THREADS 128
 #endif

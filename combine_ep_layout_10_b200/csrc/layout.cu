@@ -335,9 +335,39 @@ __device__ __forceinline__ void fill_minus_one(int32_t *dst, int64_t n) {
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
 
+// Padded layouts (capacity > 0) have every padding row in a known place,
+// [e*C + min(cnt[e], C), (e+1)*C), so helper CTAs fill them in parallel with
+// CTA 0: each counts the ids of its share of experts and writes -1 to their
+// tails.  The tails never overlap a valid row, so no ordering with CTA 0 is
+// needed.
+__device__ void small_fill_padding_tails(const LayoutArgs &a, int32_t *cnt_h) {
+    const int nh = gridDim.x - 1;
+    const int hb = blockIdx.x - 1;
+    const int e0 = (int)((int64_t)hb * a.E / nh);
+    const int e1 = (int)((int64_t)(hb + 1) * a.E / nh);
+    for (int i = threadIdx.x; i < e1 - e0; i += blockDim.x) cnt_h[i] = 0;
+    __syncthreads();
+    const int nslots = a.T * a.k;
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int e = __ldg(a.topk_idx + s);
+        if (e >= e0 && e < e1) atomicAdd(&cnt_h[e - e0], 1);
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int e = e0 + (threadIdx.x >> 5); e < e1; e += blockDim.x >> 5) {
+        const int64_t start = (int64_t)e * a.capacity + min(cnt_h[e - e0], a.capacity);
+        const int64_t end = (int64_t)(e + 1) * a.capacity;
+        for (int64_t row = start + lane; row < end; row += 32) a.src_idx[row] = -1;
+    }
+}
+
 __global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     pdl_wait_then_trigger();
+    if (blockIdx.x > 0) {  // padding helper (padded mode only)
+        small_fill_padding_tails(a, reinterpret_cast<int32_t *>(smem));
+        return;
+    }
     const int E = a.E, R = a.R;
     const int RW = (R + 31) >> 5;
     const int nslots = a.T * a.k;
@@ -446,8 +476,12 @@ __global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutArgs 
             a.out_in_rank[i] = (uint8_t)((mask_s[t * RW + (r >> 5)] >> (r & 31)) & 1u);
         }
     }
-    fill_minus_one(a.src_idx, a.n_rows);
-    __syncthreads();  // orders the -1 fill before the valid rows below
+    if (gridDim.x == 1) {
+        // Packed mode: every row starts as padding (-1); the barrier orders
+        // the fill before the valid rows are written over it below.
+        fill_minus_one(a.src_idx, a.n_rows);
+        __syncthreads();
+    }
 
     // Positions: rank inside the expert in slot order.
     const unsigned lt_mask = (1u << lane) - 1u;
@@ -529,7 +563,14 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s) {
     if (a.small) {
         const size_t smem = layout_small_smem(a);
         if ((err = ensure_dyn_smem(layout_small_kernel, smem, g_smem_small)) != cudaSuccess) return err;
-        return launch_kernel(layout_small_kernel, 1, kSmallThreads, smem, s, a);
+        // Padded mode: helper CTAs fill the padding tails, ~4096 rows each.
+        int helpers = 0;
+        if (a.capacity > 0) {
+            helpers = (int)((a.n_rows + 4095) / 4096);
+            helpers = helpers < 1 ? 1 : (helpers > 64 ? 64 : helpers);
+            if (helpers > a.E) helpers = a.E;
+        }
+        return launch_kernel(layout_small_kernel, 1 + helpers, kSmallThreads, smem, s, a);
     }
     const size_t count_smem = layout_count_smem(a);
     const size_t pos_smem = layout_pos_smem(a);

@@ -18,7 +18,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "lib", "libep_b200.so")
+#: The library this binding loads: the in-tree build, or the file named by
+#: the EP_B200_LIB environment variable (another build of the same sources).
+LIB_PATH = os.environ.get("EP_B200_LIB") or os.path.join(_HERE, "lib", "libep_b200.so")
 
 EP_OK = 0
 EP_ERR_INVALID_ARG = 1
