@@ -51,8 +51,8 @@ HBM_FALLBACK_GBS = 6650.0
 # kernel source it was taken on (stale -> reported as null).
 NCU_TRAFFIC = {
     # one "ncu --set full" capture of one launch each on the metric workload
-    ("group_limited", "combine"): {"sha": "e4aaa5203a4c74cf", "bytes": 940057856 + 73635328},
-    ("group_limited", "dispatch"): {"sha": "23a3a09c311a730d", "bytes": 117871104 + 427218944},
+    ("group_limited", "combine"): {"sha": "5dba458197e1f277", "bytes": 940058880 + 71877120},
+    ("group_limited", "dispatch"): {"sha": "557118bc734ec7e1", "bytes": 117844992 + 427099136},
 }
 
 
