@@ -77,6 +77,8 @@ def load(path: str):
         L.oracle_combine_backward.restype = i32
         L.oracle_dispatch_fp8_prequant.argtypes = [P, P, i32, i32, i32, P, P, P, i64]
         L.oracle_dispatch_fp8_prequant.restype = i32
+        L.oracle_dispatch_topk.argtypes = [P, P, i32, i32, P, i64, P, P, P]
+        L.oracle_dispatch_topk.restype = i32
     return L
 
 
@@ -241,6 +243,24 @@ def quantize_group(xg) -> tuple[np.ndarray, float]:
     s = np.zeros(1, np.float32)
     lib().oracle_quantize_group(_ptr(xb), _ptr(q), _ptr(s))
     return q, float(s[0])
+
+
+def dispatch_topk(topk_idx, w, pos: np.ndarray, n_rows: int):
+    """Per-row routing outputs of dispatch: (recv_topk_idx int32 [n_rows],
+    recv_topk_weights float32 [n_rows], recv_slot int32 [n_rows]); -1 / 0 / -1
+    on rows no slot fills."""
+    idx = np.ascontiguousarray(np.asarray(topk_idx), dtype=np.int32)
+    w = np.ascontiguousarray(np.asarray(w), dtype=np.float32)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    T, k = pos.shape
+    assert idx.shape == (T, k) and w.shape == (T, k)
+    ri = np.empty(n_rows, np.int32)
+    rw = np.empty(n_rows, np.float32)
+    rs = np.empty(n_rows, np.int32)
+    st = lib().oracle_dispatch_topk(_ptr(idx), _ptr(w), T, k, _ptr(pos), n_rows, _ptr(ri), _ptr(rw), _ptr(rs))
+    if st != OR_OK:
+        raise OracleError(st, "oracle_dispatch_topk")
+    return ri, rw, rs
 
 
 def combine(y, w: np.ndarray, pos: np.ndarray) -> np.ndarray:

@@ -496,3 +496,43 @@ int oracle_dispatch_fp8_prequant(const uint8_t *xq, const float *xs, int T, int 
     }
     return OR_OK;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Per-row routing outputs of dispatch                                        */
+/* ------------------------------------------------------------------------- */
+
+/* Besides the received rows, dispatch returns recv_topk_idx and
+ * recv_topk_weights ("DeepEP (DeepEveryParallel) Documentation", item 10).
+ * In this layout every receive row holds exactly one slot (t, j), so the
+ * per-row values are that slot's expert id topk_idx[t][j], its weight
+ * topk_w[t][j] and its flat index t*k + j.  A row that no slot fills
+ * (padding, alignment slack, rows left by unused slots) gets -1, 0.0f, -1.
+ * Any output pointer may be NULL. */
+int oracle_dispatch_topk(const int32_t *topk_idx, const float *topk_w, int T, int k,
+                         const int32_t *pos, int64_t n_rows, int32_t *recv_idx,
+                         float *recv_w, int32_t *recv_slot) {
+    if (T < 0 || k < 1 || n_rows < 0) {
+        return OR_ERR_INVALID_ARG;
+    }
+    for (int64_t r = 0; r < n_rows; ++r) {
+        if (recv_idx) recv_idx[r] = -1;
+        if (recv_w) recv_w[r] = 0.0f;
+        if (recv_slot) recv_slot[r] = -1;
+    }
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int64_t s = (int64_t)t * k + j;
+            int32_t p = pos[s];
+            if (p < 0) {
+                continue;
+            }
+            if (p >= n_rows) {
+                return OR_ERR_INVALID_ARG;
+            }
+            if (recv_idx) recv_idx[p] = topk_idx[s];
+            if (recv_w) recv_w[p] = topk_w[s];
+            if (recv_slot) recv_slot[p] = (int32_t)s;
+        }
+    }
+    return OR_OK;
+}

@@ -16,6 +16,7 @@ import test_oracle_backward as PB
 import test_oracle_dispatch_combine as PD
 import test_oracle_formats as PF
 import test_oracle_layout as PL
+import test_oracle_topk as PT
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "ep_oracle.c")
@@ -72,6 +73,20 @@ MUTANTS = [
     ("grad_y without the weight",
      "float prod = w[s] * g;", "float prod = g;",
      [(PB.test_combine_backward_vs_autograd, {"name": "tiny"})]),
+    ("per-row weight taken from the neighbouring slot",
+     "if (recv_w) recv_w[p] = topk_w[s];",
+     "if (recv_w) recv_w[p] = topk_w[s ^ 1];",
+     [(PT.test_golden_dispatch_topk, {"case": PT.TOPK["cases"][0]}),
+      (PT.test_packed_equals_stable_sort, {"name": "tiny"})]),
+    ("per-row slot id without the token",
+     "if (recv_slot) recv_slot[p] = (int32_t)s;",
+     "if (recv_slot) recv_slot[p] = (int32_t)j;",
+     [(PT.test_golden_dispatch_topk, {"case": PT.TOPK["cases"][0]}),
+      (PT.test_packed_equals_stable_sort, {"name": "tiny"})]),
+    ("padding rows keep a stale weight",
+     "        if (recv_w) recv_w[r] = 0.0f;",
+     "        if (recv_w) recv_w[r] = 1.0f;",
+     [(PT.test_golden_dispatch_topk, {"case": PT.TOPK["cases"][1]})]),
     ("grad_w missing the last channel",
      "            double dot = 0.0;\n            for (int i = 0; i < H; ++i) {",
      "            double dot = 0.0;\n            for (int i = 0; i < H - 1; ++i) {",
