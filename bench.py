@@ -657,6 +657,9 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
     d_us = timed(lambda: ep.ep_dispatch_backward(h, grad_recv, grad_x))
     c_us = timed(lambda: ep.ep_combine_backward(h, grad_out, tw_dev, y=y_dev, grad_y=grad_y,
                                                 grad_weights=grad_w))
+    # per-row routing outputs (recv_topk_idx / recv_topk_weights / slot), which
+    # a weighted expert GEMM or a per-row backward reads
+    t_us = timed(lambda: ep.ep_dispatch_topk(h, tw_dev))
     status = h.check()
     h.free()
     if status != ep.EP_OK:
@@ -664,8 +667,10 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
     V = int((idx_dev >= 0).sum().item())
     d_bytes = V * H * 2 + T * k * 4 + T * H * 2
     c_bytes = T * H * 2 + V * H * 2 + T * k * 8 + V * H * 2 + T * k * 4
+    t_bytes = rows * 4 + T * k * 4 + V * 4 + (w.E + 1) * 4 + rows * 12
     return {"dispatch_backward": {"us": d_us, "bytes": d_bytes, "gbs": d_bytes / d_us / 1e3},
-            "combine_backward": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3}}
+            "combine_backward": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3},
+            "dispatch_topk": {"us": t_us, "bytes": t_bytes, "note": "latency-bound (~1.6 MB)"}}
 
 
 def run_overlap(w, dev, ep, idx_dev, x_dev, tw_dev, y_dev, flush_l2, reps: int = 10) -> dict:

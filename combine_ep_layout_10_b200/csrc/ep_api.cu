@@ -362,6 +362,35 @@ ep_status ep_combine_backward(const ep_handle *h, const void *grad_out, const vo
     return cuda_status(launch_combine_backward(a, stream));
 }
 
+ep_status ep_dispatch_topk(const ep_handle *h, const float *topk_w, int32_t *recv_topk_idx,
+                           float *recv_topk_weights, int32_t *recv_slot, size_t recv_rows,
+                           ep_stream_t stream) {
+    if (h == nullptr) return EP_ERR_INVALID_ARG;
+    if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    if (recv_topk_weights != nullptr && h->T > 0 && (topk_w == nullptr || !aligned(topk_w, 4)))
+        return EP_ERR_INVALID_ARG;
+    if ((recv_topk_idx && !aligned(recv_topk_idx, 4)) || (recv_topk_weights && !aligned(recv_topk_weights, 4)) ||
+        (recv_slot && !aligned(recv_slot, 4)))
+        return EP_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != h->device) return EP_ERR_INVALID_ARG;
+    if (recv_topk_idx == nullptr && recv_topk_weights == nullptr && recv_slot == nullptr) return EP_OK;
+    RecvTopkArgs a{};
+    a.src_idx = h->src_idx;
+    a.pos = h->pos;
+    a.seg = h->seg;
+    a.w = recv_topk_weights != nullptr ? topk_w : nullptr;
+    a.out_idx = recv_topk_idx;
+    a.out_w = recv_topk_weights;
+    a.out_slot = recv_slot;
+    a.T = h->T; a.k = h->k; a.E = h->E;
+    a.n_rows = h->n_rows;
+    return cuda_status(launch_recv_topk(a, stream));
+}
+
 void ep_handle_free(ep_handle *h) {
     if (h == nullptr) return;
     if (h->block != nullptr) {

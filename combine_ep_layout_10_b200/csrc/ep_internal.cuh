@@ -201,6 +201,18 @@ struct CombineBwdArgs {
     int T, k, H;
 };
 
+struct RecvTopkArgs {
+    const int32_t *src_idx;  // [n_rows] (handle)
+    const int32_t *pos;      // [T, k] (handle)
+    const int32_t *seg;      // [E + 1] (handle)
+    const float *w;          // [T, k] or nullptr
+    int32_t *out_idx;        // [n_rows] or nullptr
+    float *out_w;            // [n_rows] or nullptr
+    int32_t *out_slot;       // [n_rows] or nullptr
+    int T, k, E;
+    int64_t n_rows;
+};
+
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 size_t layout_count_smem(const LayoutArgs &a);
@@ -209,6 +221,7 @@ size_t layout_pos_smem(const LayoutArgs &a);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
+cudaError_t launch_recv_topk(const RecvTopkArgs &a, cudaStream_t s);
 
 // Per-device facts, cached.
 struct DeviceInfo {

@@ -37,7 +37,7 @@ ABI_SYMBOLS = (
     "ep_status_str", "ep_max_recv_rows", "ep_layout", "ep_dispatch", "ep_combine",
     "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
     "ep_handle_check", "ep_layout_noalloc", "ep_dispatch_backward", "ep_combine_backward",
-    "ep_dispatch_ex", "ep_combine_ex",
+    "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk",
 )
 
 EP_FORMAT_BF16 = 0
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_ex.argtypes = [P, P, P, I, I, I, P, P, I64, I64, P, S, I, P]
         L.ep_dispatch_ex.restype = I
         L.ep_combine_ex.argtypes = [P, P, P, I, S, P, I, P]
+        L.ep_dispatch_topk.argtypes = [P, P, P, P, P, S, P]
+        L.ep_dispatch_topk.restype = I
         L.ep_combine_ex.restype = I
         _LIB = L
     return _LIB
@@ -320,6 +322,26 @@ def ep_combine_ex(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,
                              num_sms, _stream(stream))
     _check(st, "ep_combine_ex")
     return out
+
+
+def ep_dispatch_topk(handle: Handle, topk_weights: Optional[torch.Tensor] = None, want_idx: bool = True,
+                     want_slot: bool = True, stream=None):
+    """Per-row routing outputs of dispatch: (recv_topk_idx int32 [rows],
+    recv_topk_weights fp32 [rows] or None when topk_weights is None,
+    recv_slot int32 [rows] or None); -1 / 0 / -1 on rows no slot fills."""
+    rows = handle.num_recv_rows
+    dev = handle.device
+    ri = torch.empty(rows, dtype=torch.int32, device=dev) if want_idx else None
+    rw = torch.empty(rows, dtype=torch.float32, device=dev) if topk_weights is not None else None
+    rs = torch.empty(rows, dtype=torch.int32, device=dev) if want_slot else None
+    st = lib().ep_dispatch_topk(handle.ptr,
+                                _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                         (handle.num_tokens, handle.num_topk)),
+                                _dev_ptr(ri, torch.int32, "recv_topk_idx"),
+                                _dev_ptr(rw, torch.float32, "recv_topk_weights"),
+                                _dev_ptr(rs, torch.int32, "recv_slot"), rows, _stream(stream))
+    _check(st, "ep_dispatch_topk")
+    return ri, rw, rs
 
 
 def ep_dispatch_backward(handle: Handle, grad_recv: torch.Tensor, grad_x: Optional[torch.Tensor] = None,

@@ -216,6 +216,28 @@ ep_status ep_combine_ex(const ep_handle *handle, const void *y, const float *top
                         int hidden, size_t recv_rows, void *combined_x, int num_sms,
                         ep_stream_t stream);
 
+/* Per-row routing outputs of dispatch: the pages' recv_topk_idx and
+ * recv_topk_weights (docsearch item 10: dispatch returns them beside recv_x),
+ * plus the slot each row came from.  Every receive row of this layout holds
+ * one slot (t, j); for each row r < num_recv_rows of the handle:
+ *   r filled by slot (t, j):  recv_topk_idx[r]     = topk_idx[t][j]  (the expert whose segment holds r)
+ *                             recv_topk_weights[r] = topk_weights[t][j]  (bit copy)
+ *                             recv_slot[r]         = t * k + j  (so t = recv_slot / k = src_idx[r])
+ *   r filled by no slot:      -1, 0.0f, -1
+ *   topk_weights: device fp32 [T, k]; read only when recv_topk_weights is
+ *     not NULL (then it must not be NULL).
+ *   recv_topk_idx, recv_topk_weights, recv_slot: device [recv_rows] int32 /
+ *     fp32 / int32, 4-byte aligned, each may be NULL (nothing to do when all
+ *     are).  All num_recv_rows rows are written, padding rows included; rows
+ *     past num_recv_rows are not touched.
+ *   recv_rows: length of those buffers, >= num_recv_rows of the handle.
+ * Asynchronous, no allocation, no host synchronisation (capturable in a CUDA
+ * graph with a kept handle).  If the layout found a data error the values
+ * are unspecified but every write stays inside the buffers. */
+ep_status ep_dispatch_topk(const ep_handle *handle, const float *topk_weights,
+                           int32_t *recv_topk_idx, float *recv_topk_weights, int32_t *recv_slot,
+                           size_t recv_rows, ep_stream_t stream);
+
 /* Release a handle.  Its device memory is freed stream-ordered on the stream
  * that created it (cudaFreeAsync); work that uses the handle on other streams
  * must be ordered before that stream's current position by the caller.
