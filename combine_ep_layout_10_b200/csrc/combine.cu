@@ -17,6 +17,11 @@
 // FMA chain in slot order and stores 16 bytes.  With no weights (w == nullptr)
 // every weight is 1: fmaf(1, y, acc) is the correctly rounded acc + y, which
 // makes the same kernel the backward of dispatch (sum of the k row gradients).
+// Threads j < k resolve the token's k source rows to pointers first: row
+// pos[t][j] of the local y, or, when the ranks are real GPUs (PEER), row d.y
+// of rank d.x's expert outputs, d = dst[t][j] of the plan, read through that
+// rank's mapping in this process (NVLink peer loads; y is not written by
+// anyone while the combine runs).
 #include <cuda_bf16.h>
 
 #include "ep_internal.cuh"
@@ -68,9 +73,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
-template <int VPT, bool LOOP>
+template <int VPT, bool LOOP, bool PEER>
 __global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(CombineArgs a) {
-    __shared__ int32_t p_s[kMaxTopk];
+    __shared__ const uint8_t *src_s[kMaxTopk];
     __shared__ float w_s[kMaxTopk];
     pdl_wait_then_trigger();
     const size_t row_bytes = (size_t)a.H * 2;
@@ -82,8 +87,17 @@ __global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(
     const int t = b / a.blocks_per_token;
     const int cb = b - t * a.blocks_per_token;
     if (threadIdx.x < a.k) {
-        p_s[threadIdx.x] = __ldg(a.pos + (int64_t)t * a.k + threadIdx.x);
-        w_s[threadIdx.x] = a.w != nullptr ? __ldg(a.w + (int64_t)t * a.k + threadIdx.x) : 1.0f;
+        const int64_t s = (int64_t)t * a.k + threadIdx.x;
+        const uint8_t *src = nullptr;
+        if (PEER) {
+            const int2 d = __ldg(a.src + s);
+            if (d.x >= 0) src = a.peer_y[d.x] + (size_t)d.y * row_bytes;
+        } else {
+            const int p = __ldg(a.pos + s);
+            if (p >= 0) src = a.y + (size_t)p * row_bytes;
+        }
+        src_s[threadIdx.x] = src;
+        w_s[threadIdx.x] = a.w != nullptr ? __ldg(a.w + s) : 1.0f;
     }
     __syncthreads();
 
@@ -97,14 +111,14 @@ __global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(
 #pragma unroll
             for (int jj = 0; jj < kLoadBatch; ++jj) {
                 const int j = j0 + jj;
-                const int p = (j < a.k) ? p_s[j] : -1;
-                if (p >= 0) r[jj] = ld_stream_v4(a.y + (size_t)p * row_bytes + (size_t)v * 16);
+                const uint8_t *src = (j < a.k) ? src_s[j] : nullptr;
+                if (src != nullptr) r[jj] = ld_stream_v4(src + (size_t)v * 16);
             }
 #pragma unroll
             for (int jj = 0; jj < kLoadBatch; ++jj) {
                 const int j = j0 + jj;
-                const int p = (j < a.k) ? p_s[j] : -1;
-                if (p >= 0) fma8(acc, w_s[j], r[jj]);
+                const uint8_t *src = (j < a.k) ? src_s[j] : nullptr;
+                if (src != nullptr) fma8(acc, w_s[j], r[jj]);
             }
         }
         uint4 o;
@@ -115,22 +129,23 @@ __global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(
         st_out_v4(a.out + (size_t)t * row_bytes + (size_t)v * 16, o);
     }
     if (!LOOP) break;
-    __syncthreads();  // p_s / w_s are rewritten for the next pair
+    __syncthreads();  // src_s / w_s are rewritten for the next pair
     }
 }
 
-}  // namespace
-
-cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
+template <bool PEER>
+cudaError_t launch_combine_impl(const CombineArgs &a, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     long long blocks = (long long)a.T * a.blocks_per_token;
     if ((long long)a.blocks_per_token * a.vpt * kCombineThreads < a.nvec)
         return cudaErrorInvalidConfiguration;
     const bool loop = a.num_sms > 0;
     void (*kernel)(CombineArgs) = nullptr;
-    if (a.vpt == 1) kernel = loop ? combine_kernel<1, true> : combine_kernel<1, false>;
-    if (a.vpt == 2) kernel = loop ? combine_kernel<2, true> : combine_kernel<2, false>;
-    if (a.vpt == 4) kernel = loop ? combine_kernel<4, true> : combine_kernel<4, false>;
+    if (a.vpt == 1) kernel = loop ? combine_kernel<1, true, PEER> : combine_kernel<1, false, PEER>;
+    if (!PEER) {  // wider vectors per thread: a tuning option of the local path only
+        if (a.vpt == 2) kernel = loop ? combine_kernel<2, true, false> : combine_kernel<2, false, false>;
+        if (a.vpt == 4) kernel = loop ? combine_kernel<4, true, false> : combine_kernel<4, false, false>;
+    }
     if (kernel == nullptr) return cudaErrorInvalidConfiguration;
     if (loop) {
         int per_sm = 0;
@@ -141,5 +156,11 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
     }
     return launch_kernel(kernel, (unsigned)blocks, kCombineThreads, 0, s, a);
 }
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) { return launch_combine_impl<false>(a, s); }
+
+cudaError_t launch_combine_peer(const CombineArgs &a, cudaStream_t s) { return launch_combine_impl<true>(a, s); }
 
 }  // namespace ep

@@ -23,6 +23,10 @@
 //     the group's first lane copies the scale.
 // FP8 scales are written at p * s_row + g * s_grp (row-major [rows, H/128],
 // or column-major with a caller-chosen leading dimension for FP8 GEMMs).
+// Threads j < k resolve the block's k destination rows to pointers first:
+// row pos[t][j] of the local receive buffer, or, when the ranks are real GPUs
+// (PEER), row d.y of rank d.x's receive buffer, d = dst[t][j] of the plan,
+// reached through that rank's mapping in this process (NVLink peer stores).
 // A TMA variant (bulk load into a shared ring, k bulk stores from shared
 // memory) was measured slower on this path: bulk stores of scattered 7-14 KB
 // rows sustain less write bandwidth on B200 than plain 16-byte stores.
@@ -66,12 +70,40 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     f[7] = bf16_bits_to_f32(v.w >> 16);
 }
 
+// Receive-row pointers of token t's k slots (nullptr for a slot without a
+// row), written to shared memory by threads j < k.
+template <bool PEER>
+__device__ __forceinline__ void slot_rows(const DispatchArgs &a, int t, size_t row_bytes, uint8_t **row_s,
+                                          float **srow_s) {
+    const int j = threadIdx.x;
+    if (j >= a.k) return;
+    const int64_t s = (int64_t)t * a.k + j;
+    uint8_t *row = nullptr;
+    float *srow = nullptr;
+    if (PEER) {
+        const int2 d = __ldg(a.dst + s);
+        if (d.x >= 0) {
+            row = a.peer_recv[d.x] + (size_t)d.y * row_bytes;
+            if (a.peer_scales != nullptr) srow = a.peer_scales[d.x] + (int64_t)d.y * a.s_row;
+        }
+    } else {
+        const int p = __ldg(a.pos + s);
+        if (p >= 0) {
+            row = a.recv + (size_t)p * row_bytes;
+            if (a.scales != nullptr) srow = a.scales + (int64_t)p * a.s_row;
+        }
+    }
+    row_s[j] = row;
+    srow_s[j] = srow;
+}
+
 // The kernels take one (token, chunk) unit per block; when the caller caps
 // the grid (num_sms) the LOOP instantiation walks the units with a grid stride.
 
-template <bool LOOP>
+template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
-    __shared__ int32_t p_s[kMaxTopk];
+    __shared__ uint8_t *row_s[kMaxTopk];
+    __shared__ float *srow_s[kMaxTopk];
     pdl_wait_then_trigger();
     const int tid = threadIdx.x;
     const bool leader = (tid & 7) == 0;
@@ -80,7 +112,6 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
         const int t = u / a.nchunks;
         const int ch0 = (u - t * a.nchunks) * a.chunk;
         const int chn = min(a.chunk, a.H - ch0);
-        if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
         const int ch = ch0 + tid * 16;
         const bool act = tid * 16 < chn;
         uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
@@ -89,6 +120,7 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
             v0 = ld_nc_v4(src);
             v1 = ld_nc_v4(src + 16);
         }
+        slot_rows<PEER>(a, t, (size_t)a.H, row_s, srow_s);  // after the x loads are in flight
         __syncthreads();
         float f[16];
         unpack8(v0, f);
@@ -119,21 +151,22 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
             }
             const int g = ch / 128;
             for (int j = 0; j < a.k; ++j) {
-                const int p = p_s[j];
-                if (p < 0) continue;
-                st_row_v4(a.recv + (int64_t)p * a.H + ch, q16);
-                if (leader) a.scales[(int64_t)p * a.s_row + (int64_t)g * a.s_grp] = scale;
+                uint8_t *row = row_s[j];
+                if (row == nullptr) continue;
+                st_row_v4(row + ch, q16);
+                if (leader) srow_s[j][(int64_t)g * a.s_grp] = scale;
             }
         }
         if (!LOOP) break;
-        __syncthreads();  // p_s is rewritten by the next unit
+        __syncthreads();  // row_s is rewritten by the next unit
     }
 }
 
 // Pre-quantised FP8 input: codes and scales are copied, not recomputed.
-template <bool LOOP>
+template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) {
-    __shared__ int32_t p_s[kMaxTopk];
+    __shared__ uint8_t *row_s[kMaxTopk];
+    __shared__ float *srow_s[kMaxTopk];
     pdl_wait_then_trigger();
     const int tid = threadIdx.x;
     const bool leader = (tid & 7) == 0;
@@ -143,7 +176,6 @@ __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) 
         const int t = u / a.nchunks;
         const int ch0 = (u - t * a.nchunks) * a.chunk;
         const int chn = min(a.chunk, a.H - ch0);
-        if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
         const int ch = ch0 + tid * 16;
         const bool act = tid * 16 < chn;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -152,24 +184,26 @@ __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) 
             v = ld_nc_v4(a.x + (int64_t)t * a.H + ch);
             if (leader) scale = __ldg(a.x_scales + (int64_t)t * G_row + ch / 128);
         }
+        slot_rows<PEER>(a, t, (size_t)a.H, row_s, srow_s);  // after the x loads are in flight
         __syncthreads();
         if (act) {
             const int g = ch / 128;
             for (int j = 0; j < a.k; ++j) {
-                const int p = p_s[j];
-                if (p < 0) continue;
-                st_row_v4(a.recv + (int64_t)p * a.H + ch, v);
-                if (leader) a.scales[(int64_t)p * a.s_row + (int64_t)g * a.s_grp] = scale;
+                uint8_t *row = row_s[j];
+                if (row == nullptr) continue;
+                st_row_v4(row + ch, v);
+                if (leader) srow_s[j][(int64_t)g * a.s_grp] = scale;
             }
         }
         if (!LOOP) break;
-        __syncthreads();  // p_s is rewritten by the next unit
+        __syncthreads();  // row_s is rewritten by the next unit
     }
 }
 
-template <bool LOOP>
+template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchArgs a) {
-    __shared__ int32_t p_s[kMaxTopk];
+    __shared__ uint8_t *row_s[kMaxTopk];
+    __shared__ float *srow_s[kMaxTopk];
     pdl_wait_then_trigger();
     const int tid = threadIdx.x;
     // One unit per block unless the grid is capped (LOOP): then a grid stride.
@@ -177,7 +211,6 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchArgs a) {
         const int t = u / a.nchunks;
         const int ch0 = (u - t * a.nchunks) * a.chunk;
         const int chn = min(a.chunk, a.H - ch0);
-        if (tid < a.k) p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
         // Two 16-byte vectors per thread, a block apart, so that every warp-wide
         // load and store covers 512 contiguous bytes.
         const int nv = chn / 8;
@@ -187,32 +220,34 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchArgs a) {
         const uint8_t *src = a.x + ((int64_t)t * a.H + ch0) * 2;
         if (act0) v0 = ld_nc_v4(src + (size_t)u0 * 16);
         if (act1) v1 = ld_nc_v4(src + (size_t)u1 * 16);
+        slot_rows<PEER>(a, t, (size_t)a.H * 2, row_s, srow_s);  // after the x loads are in flight
         __syncthreads();
         if (act0) {
             for (int j = 0; j < a.k; ++j) {
-                const int p = p_s[j];
-                if (p < 0) continue;
-                uint8_t *dst = a.recv + ((int64_t)p * a.H + ch0) * 2;
+                uint8_t *row = row_s[j];
+                if (row == nullptr) continue;
+                uint8_t *dst = row + (size_t)ch0 * 2;
                 st_row_v4(dst + (size_t)u0 * 16, v0);
                 if (act1) st_row_v4(dst + (size_t)u1 * 16, v1);
             }
         }
         if (!LOOP) break;
-        __syncthreads();  // p_s is rewritten by the next unit
+        __syncthreads();  // row_s is rewritten by the next unit
     }
 }
 
-}  // namespace
-
-cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
+template <bool PEER>
+cudaError_t launch_dispatch_impl(const DispatchArgs &a, cudaStream_t st) {
     if (a.nunits == 0) return cudaSuccess;
     // One block per unit, one thread per 16 channels (chunk <= 8192 -> <= 512 threads).
     const int threads = (((a.chunk + 15) / 16 + 31) / 32) * 32;
     const bool loop = a.num_sms > 0;
     void (*kernel)(DispatchArgs) =
-        a.mode == kDispatchQuantFp8 ? (loop ? dispatch_fp8_kernel<true> : dispatch_fp8_kernel<false>)
-        : a.mode == kDispatchCopyFp8 ? (loop ? dispatch_fp8_copy_kernel<true> : dispatch_fp8_copy_kernel<false>)
-                                     : (loop ? dispatch_bf16_kernel<true> : dispatch_bf16_kernel<false>);
+        a.mode == kDispatchQuantFp8
+            ? (loop ? dispatch_fp8_kernel<true, PEER> : dispatch_fp8_kernel<false, PEER>)
+        : a.mode == kDispatchCopyFp8
+            ? (loop ? dispatch_fp8_copy_kernel<true, PEER> : dispatch_fp8_copy_kernel<false, PEER>)
+            : (loop ? dispatch_bf16_kernel<true, PEER> : dispatch_bf16_kernel<false, PEER>);
     int grid = a.nunits;
     if (loop) {
         int per_sm = 0;
@@ -223,5 +258,11 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
     }
     return launch_kernel(kernel, (unsigned)grid, threads, 0, st, a);
 }
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t st) { return launch_dispatch_impl<false>(a, st); }
+
+cudaError_t launch_dispatch_peer(const DispatchArgs &a, cudaStream_t st) { return launch_dispatch_impl<true>(a, st); }
 
 }  // namespace ep

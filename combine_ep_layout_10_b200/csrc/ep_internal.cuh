@@ -106,6 +106,23 @@ struct ep_handle {
     uint32_t *err;           // [1] device error word
 };
 
+// The opaque multi-rank plan of the ABI: where every local slot goes on
+// which rank, and this rank's receive segments.  Host struct; the arrays are
+// device memory carved out of one stream-ordered allocation.
+struct ep_plan {
+    int T, k, E, world, rank, epr, align, capacity;
+    int64_t recv_rows;       // rows of every rank's receive buffer
+    int device;
+    cudaStream_t stream;
+    void *block;
+    int2 *dst;               // [T*k] (owner rank, row in its receive buffer), (-1, -1) if none
+    int32_t *pre;            // [E] slots of lower source ranks per expert (scratch)
+    int32_t *offs;           // [E] row of this rank's first slot of each expert (scratch)
+    int32_t *recv_seg;       // [epr+1] segment starts of this rank's experts in its receive buffer
+    int32_t *recv_cnt;       // [epr] slots routed to each of this rank's experts (all sources)
+    uint32_t *err;           // [1] device error word
+};
+
 namespace ep {
 
 __host__ __device__ constexpr int align4(int n) { return (n + 3) & ~3; }
@@ -177,6 +194,10 @@ struct DispatchArgs {
     int chunk;               // channels per work unit
     int nchunks;             // units per token
     int nunits;              // T * nchunks (< 2^31, checked on the host)
+    // Multi-rank (peer) addressing, used instead of pos / recv / scales:
+    const int2 *dst;                 // [T, k] (rank, row) of each slot, rank -1 if none
+    uint8_t *const *peer_recv;       // [world] device pointers to every rank's receive buffer
+    float *const *peer_scales;       // [world] ... scale buffers (FP8), or nullptr
 };
 
 struct CombineArgs {
@@ -189,6 +210,9 @@ struct CombineArgs {
     int vpt;                 // vectors per thread: 1, 2 or 4
     int blocks_per_token;    // ceil(nvec / (128 * vpt))
     int num_sms;             // 0: one block per (token, vector block); else grid capped
+    // Multi-rank (peer) addressing, used instead of pos / y:
+    const int2 *src;                 // [T, k] (rank, row) of each slot's expert output, rank -1 if none
+    const uint8_t *const *peer_y;    // [world] device pointers to every rank's expert outputs
 };
 
 struct CombineBwdArgs {
@@ -213,6 +237,51 @@ struct RecvTopkArgs {
     int64_t n_rows;
 };
 
+// Exclusive scan of one value per thread over the block (blockDim.x <= 1024);
+// returns the exclusive prefix and writes the block total to *total.
+// warp_s: 33 words of shared memory.  Every thread of the block must call it.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t *total, int32_t *warp_s) {
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    int32_t incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t n = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += n;
+    }
+    if (lane == 31) warp_s[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int32_t w = (lane < nwarps) ? warp_s[lane] : 0;
+        int32_t wi = w;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t n = __shfl_up_sync(0xffffffffu, wi, d);
+            if (lane >= d) wi += n;
+        }
+        warp_s[lane] = wi - w;
+        if (lane == 31) warp_s[32] = wi;
+    }
+    __syncthreads();
+    const int32_t excl = warp_s[warp] + incl - v;
+    *total = warp_s[32];
+    __syncthreads();
+    return excl;
+}
+
+struct PlanArgs {
+    const int32_t *topk_idx;   // [T, k] this rank's ids
+    const int32_t *pos;        // [T, k] local layout (packed, alignment 1)
+    const int32_t *seg;        // [E + 1] local layout
+    const int32_t *counts;     // [world, E] every rank's per-expert slot counts
+    int T, k, E, world, rank, epr, align, capacity;
+    int64_t recv_rows;
+    int2 *dst;
+    int32_t *pre, *offs, *recv_seg, *recv_cnt;
+    uint32_t *err;
+};
+
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 size_t layout_count_smem(const LayoutArgs &a);
@@ -222,6 +291,10 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
 cudaError_t launch_recv_topk(const RecvTopkArgs &a, cudaStream_t s);
+cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
+// Peer-addressed variants of dispatch and combine (DispatchArgs::dst, CombineArgs::src).
+cudaError_t launch_dispatch_peer(const DispatchArgs &a, cudaStream_t s);
+cudaError_t launch_combine_peer(const CombineArgs &a, cudaStream_t s);
 
 // Per-device facts, cached.
 struct DeviceInfo {

@@ -31,38 +31,6 @@ namespace {
 constexpr int kCountThreads = 256;
 constexpr int kPosThreads = 256;
 
-// Exclusive scan of one value per thread over the block (blockDim.x <= 1024);
-// returns the exclusive prefix and writes the block total to *total.
-__device__ int32_t block_exclusive_scan(int32_t v, int32_t *total, int32_t *warp_s) {
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int nwarps = (blockDim.x + 31) >> 5;
-    int32_t incl = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int32_t n = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += n;
-    }
-    if (lane == 31) warp_s[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int32_t w = (lane < nwarps) ? warp_s[lane] : 0;
-        int32_t wi = w;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int32_t n = __shfl_up_sync(0xffffffffu, wi, d);
-            if (lane >= d) wi += n;
-        }
-        warp_s[lane] = wi - w;
-        if (lane == 31) warp_s[32] = wi;
-    }
-    __syncthreads();
-    const int32_t excl = warp_s[warp] + incl - v;
-    *total = warp_s[32];
-    __syncthreads();
-    return excl;
-}
-
 // Copy n int32 words global -> shared (16-byte vectors when both are aligned).
 __device__ __forceinline__ void load_words(int32_t *dst, const int32_t *src, int n) {
     if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {

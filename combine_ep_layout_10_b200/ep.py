@@ -38,7 +38,12 @@ ABI_SYMBOLS = (
     "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
     "ep_handle_check", "ep_layout_noalloc", "ep_dispatch_backward", "ep_combine_backward",
     "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk",
+    "ep_peer_max_recv_rows", "ep_plan_create", "ep_plan_free", "ep_plan_export", "ep_plan_recv_rows_host",
+    "ep_plan_check", "ep_peers_create", "ep_peers_free", "ep_dispatch_peer", "ep_combine_peer",
+    "ep_ipc_export", "ep_ipc_import", "ep_ipc_release",
 )
+
+EP_IPC_HANDLE_BYTES = 64
 
 EP_FORMAT_BF16 = 0
 EP_FORMAT_E4M3 = 1
@@ -102,6 +107,33 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_topk.argtypes = [P, P, P, P, P, S, P]
         L.ep_dispatch_topk.restype = I
         L.ep_combine_ex.restype = I
+        I64, U64 = ctypes.c_int64, ctypes.c_uint64
+        L.ep_peer_max_recv_rows.argtypes = [I64, I, I, I, I, I]
+        L.ep_peer_max_recv_rows.restype = S
+        L.ep_plan_create.argtypes = [P, P, P, I, I, I, I, S, ctypes.POINTER(P), P]
+        L.ep_plan_create.restype = I
+        L.ep_plan_free.argtypes = [P]
+        L.ep_plan_free.restype = None
+        L.ep_plan_export.argtypes = [P, P, P, P, P]
+        L.ep_plan_export.restype = I
+        L.ep_plan_recv_rows_host.argtypes = [P, ctypes.POINTER(I64), P]
+        L.ep_plan_recv_rows_host.restype = I
+        L.ep_plan_check.argtypes = [P, P]
+        L.ep_plan_check.restype = I
+        L.ep_peers_create.argtypes = [I, P, P, P, S, ctypes.POINTER(P)]
+        L.ep_peers_create.restype = I
+        L.ep_peers_free.argtypes = [P]
+        L.ep_peers_free.restype = None
+        L.ep_dispatch_peer.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.ep_dispatch_peer.restype = I
+        L.ep_combine_peer.argtypes = [P, P, P, I, P, I, P]
+        L.ep_combine_peer.restype = I
+        L.ep_ipc_export.argtypes = [P, P, ctypes.POINTER(U64)]
+        L.ep_ipc_export.restype = I
+        L.ep_ipc_import.argtypes = [P, U64, ctypes.POINTER(P)]
+        L.ep_ipc_import.restype = I
+        L.ep_ipc_release.argtypes = [P, U64]
+        L.ep_ipc_release.restype = I
         _LIB = L
     return _LIB
 
@@ -408,3 +440,163 @@ def ep_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_ranks: int,
         _dev_ptr(rank_off, torch.int32, "rank_off", (num_ranks + 1,)),
         _dev_ptr(error_word, torch.int32, "error_word", (1,)), _stream(stream))
     _check(st, "ep_layout_noalloc")
+
+
+# ---------------------------------------------------------------------------
+# Expert parallelism across GPUs (one process per GPU)
+# ---------------------------------------------------------------------------
+
+def ep_peer_max_recv_rows(total_tokens: int, num_topk: int, num_experts: int, world: int,
+                          expert_alignment: int = 1, capacity: int = 0) -> int:
+    return int(lib().ep_peer_max_recv_rows(total_tokens, num_topk, num_experts, world, expert_alignment,
+                                           capacity))
+
+
+class Plan:
+    """Owner of an ep_plan*: the (rank, row) of every local slot on its owner."""
+
+    def __init__(self, ptr: ctypes.c_void_p, device, num_tokens: int, num_topk: int, num_experts: int,
+                 rank: int, world: int):
+        self._ptr = ptr
+        self.device = device
+        self.num_tokens, self.num_topk, self.num_experts = num_tokens, num_topk, num_experts
+        self.rank, self.world = rank, world
+        self.experts_per_rank = num_experts // world
+
+    @property
+    def ptr(self) -> ctypes.c_void_p:
+        if self._ptr is None:
+            raise RuntimeError("plan already freed")
+        return self._ptr
+
+    def export(self, stream=None) -> dict:
+        """Device copies of dst [T,k,2], recv_seg [E/W+1], recv_counts [E/W]."""
+        dev = self.device
+        dst = torch.empty(self.num_tokens, self.num_topk, 2, dtype=torch.int32, device=dev)
+        seg = torch.empty(self.experts_per_rank + 1, dtype=torch.int32, device=dev)
+        cnt = torch.empty(self.experts_per_rank, dtype=torch.int32, device=dev)
+        _check(lib().ep_plan_export(self.ptr, _dev_ptr(dst, None, "dst"), _dev_ptr(seg, None, "recv_seg"),
+                                    _dev_ptr(cnt, None, "recv_counts"), _stream(stream)), "ep_plan_export")
+        return {"dst": dst, "recv_seg": seg, "recv_counts": cnt}
+
+    def recv_rows_host(self, stream=None) -> int:
+        n = ctypes.c_int64(0)
+        _check(lib().ep_plan_recv_rows_host(self.ptr, ctypes.byref(n), _stream(stream)), "ep_plan_recv_rows_host")
+        return int(n.value)
+
+    def check(self, stream=None) -> int:
+        return int(lib().ep_plan_check(self.ptr, _stream(stream)))
+
+    def free(self) -> None:
+        if self._ptr is not None:
+            lib().ep_plan_free(self._ptr)
+            self._ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def ep_plan_create(local: Handle, topk_idx: torch.Tensor, all_counts: torch.Tensor, rank: int, world: int,
+                   recv_rows: int, expert_alignment: int = 1, capacity: int = 0, stream=None) -> Plan:
+    """Plan of this rank from its local layout handle (made with num_ranks =
+    world, alignment 1, capacity 0) and the all-gathered counts [world, E]."""
+    out = ctypes.c_void_p()
+    T, k = local.num_tokens, local.num_topk
+    st = lib().ep_plan_create(local.ptr, _dev_ptr(topk_idx, torch.int32, "topk_idx", (T, k)),
+                              _dev_ptr(all_counts, torch.int32, "all_counts", (world, local.num_experts)),
+                              rank, world, expert_alignment, capacity, recv_rows, ctypes.byref(out),
+                              _stream(stream))
+    _check(st, "ep_plan_create")
+    return Plan(out, topk_idx.device, T, k, local.num_experts, rank, world)
+
+
+def _ptr_array(ptrs):
+    arr = (ctypes.c_void_p * len(ptrs))()
+    for i, p in enumerate(ptrs):
+        arr[i] = int(p.data_ptr()) if isinstance(p, torch.Tensor) else int(p)
+    return arr
+
+
+class Peers:
+    """Owner of an ep_peers*: every rank's buffers as addressed from this process."""
+
+    def __init__(self, world: int, recv_x, recv_scales, y, recv_rows: int):
+        out = ctypes.c_void_p()
+        st = lib().ep_peers_create(world, _ptr_array(recv_x),
+                                   _ptr_array(recv_scales) if recv_scales is not None else None,
+                                   _ptr_array(y) if y is not None else None, recv_rows, ctypes.byref(out))
+        _check(st, "ep_peers_create")
+        self._ptr = out
+        self.world = world
+        self.recv_rows = recv_rows
+
+    @property
+    def ptr(self) -> ctypes.c_void_p:
+        if self._ptr is None:
+            raise RuntimeError("peer table already freed")
+        return self._ptr
+
+    def free(self) -> None:
+        if self._ptr is not None:
+            lib().ep_peers_free(self._ptr)
+            self._ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def ep_dispatch_peer(plan: Plan, peers: Peers, x: torch.Tensor, use_fp8: bool,
+                     x_scales: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None) -> None:
+    """Stores every local token's rows (BF16, fused FP8, or pre-quantised FP8
+    when x is float8_e4m3fn with x_scales) into the owners' receive buffers."""
+    T, H = x.shape
+    in_fp8 = x.dtype == torch.float8_e4m3fn
+    if in_fp8 and not use_fp8:
+        raise ValueError("FP8 input needs FP8 output")
+    st = lib().ep_dispatch_peer(plan.ptr, peers.ptr, _dev_ptr(x, x.dtype, "x", (plan.num_tokens, H)),
+                                _dev_ptr(x_scales, torch.float32, "x_scales"), H,
+                                EP_FORMAT_E4M3 if in_fp8 else EP_FORMAT_BF16,
+                                EP_FORMAT_E4M3 if use_fp8 else EP_FORMAT_BF16, num_sms, _stream(stream))
+    _check(st, "ep_dispatch_peer")
+
+
+def ep_combine_peer(plan: Plan, peers: Peers, topk_weights: Optional[torch.Tensor], hidden: int,
+                    out: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None) -> torch.Tensor:
+    """[T, H] bf16: each local token's weighted sum of its expert outputs read
+    from the owners' y buffers (topk_weights None: unit weights)."""
+    if out is None:
+        out = torch.empty(plan.num_tokens, hidden, dtype=torch.bfloat16, device=plan.device)
+    st = lib().ep_combine_peer(plan.ptr, peers.ptr,
+                               _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                        (plan.num_tokens, plan.num_topk)),
+                               hidden, _dev_ptr(out, torch.bfloat16, "out", (plan.num_tokens, hidden)),
+                               num_sms, _stream(stream))
+    _check(st, "ep_combine_peer")
+    return out
+
+
+def ipc_export(t: torch.Tensor):
+    """(64-byte handle, offset) of the allocation holding t, for another process."""
+    h = ctypes.create_string_buffer(EP_IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    _check(lib().ep_ipc_export(_dev_ptr(t, None, "t"), h, ctypes.byref(off)), "ep_ipc_export")
+    return h.raw, int(off.value)
+
+
+def ipc_import(handle: bytes, offset: int) -> int:
+    """Device address, in this process, of another process's exported buffer."""
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle must be %d bytes" % EP_IPC_HANDLE_BYTES)
+    out = ctypes.c_void_p()
+    _check(lib().ep_ipc_import(handle, offset, ctypes.byref(out)), "ep_ipc_import")
+    return int(out.value)
+
+
+def ipc_release(ptr: int, offset: int) -> None:
+    _check(lib().ep_ipc_release(ctypes.c_void_p(ptr), offset), "ep_ipc_release")

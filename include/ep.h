@@ -313,6 +313,123 @@ ep_status ep_layout_noalloc(const int32_t *topk_idx, int num_tokens, int num_top
                             int32_t *seg, int32_t *rank_off, uint32_t *error_word,
                             ep_stream_t stream);
 
+/* ========================================================================= *
+ * Expert parallelism across GPUs (one process per GPU, W ranks)              *
+ * ========================================================================= *
+ *
+ * The pages' dispatch sends every token to its experts on all ranks and
+ * combine returns the expert outputs to the rank the token came from
+ * (news.hada.io "Patrones de uso en entrenamiento, prefill y decoding";
+ * docsearch item 10).  Here rank r of W owns experts [r*E/W, (r+1)*E/W), and
+ * its receive buffer holds exactly the rows the single-GPU layout would give
+ * rank r for all ranks' tokens concatenated in rank order: segment by
+ * segment for its experts (packed with expert_alignment, or `capacity` rows
+ * each), inside a segment by (source rank, source token, slot).
+ *
+ * One step, on every rank, all on one stream:
+ *   1. ep_layout(local topk_idx, E, R = W, alignment 1, capacity 0) with
+ *      num_tokens_per_expert -> counts[E];
+ *   2. all-gather counts into all_counts[W][E] (e.g. NCCL; the caller's);
+ *   3. ep_plan_create(...)  -- where each local slot goes, rank and row;
+ *   4. ep_dispatch_peer(...) -- stores straight into the owners' buffers;
+ *   5. a barrier collective (every rank's stores are complete before any
+ *      rank reads its receive buffer), then the expert computation writes y;
+ *   6. a barrier collective (every y complete), then ep_combine_peer(...),
+ *      which reads the y rows from the owners' buffers.
+ * The all-gather of the next step orders that step's stores after this
+ * step's reads on every rank.  No kernel waits on another rank: ordering is
+ * the caller's collectives (a rank that does not arrive shows up as a
+ * collective timeout on the host, never as a spinning GPU).
+ * A routing that does not change reuses the plan (cached handle, item 3).
+ *
+ * Peer memory: every rank's receive / scale / expert-output buffers must be
+ * addressable from this process (ep_ipc_export / ep_ipc_import, or any other
+ * mapping); only plain loads and stores reach them (no multicast). */
+
+/* Rows a rank may receive: total_tokens (all ranks) * k, plus
+ * (E/W) * (expert_alignment - 1) of alignment slack; (E/W) * capacity when
+ * capacity > 0.  Host only, pure; 0 for invalid arguments. */
+size_t ep_peer_max_recv_rows(int64_t total_tokens, int num_topk, int num_experts, int world,
+                             int expert_alignment, int capacity);
+
+typedef struct ep_plan ep_plan;
+
+/* Plan of one rank for one routing.
+ *   local: this rank's layout handle, made with num_ranks == world,
+ *     expert_alignment 1 and capacity 0 (EP_ERR_INVALID_ARG otherwise); the
+ *     plan reads its positions and segments now and keeps no reference.
+ *   topk_idx: device int32 [T, k], the ids the local layout was made from.
+ *   all_counts: device int32 [world, E]; row s = rank s's
+ *     num_tokens_per_expert (every rank passes the same matrix).
+ *   rank, world: this rank and the group size.
+ *   expert_alignment, capacity: the receive layout, as in ep_layout (the same
+ *     on every rank).
+ *   recv_rows: rows of every rank's receive buffer (the same on every rank),
+ *     < 2^31; ep_peer_max_recv_rows() rows always suffice.
+ * Writes *out; the plan owns one stream-ordered device allocation, freed by
+ * ep_plan_free.  A slot whose row would fall past recv_rows or past a padded
+ * expert's capacity gets no row and sets the plan's error word
+ * (ep_plan_check -> EP_ERR_CAPACITY); no call ever writes outside a buffer. */
+ep_status ep_plan_create(const ep_handle *local, const int32_t *topk_idx, const int32_t *all_counts,
+                         int rank, int world, int expert_alignment, int capacity, size_t recv_rows,
+                         ep_plan **out, ep_stream_t stream);
+void ep_plan_free(ep_plan *plan);
+
+/* Copies of the plan (device-to-device, async; any destination may be NULL):
+ *   dst: int32 [T, k, 2] (owner rank, row in the owner's receive buffer) of
+ *     every local slot, (-1, -1) for a slot without a row;
+ *   recv_seg: int32 [E/W + 1] segment starts of this rank's experts in its
+ *     own receive buffer (recv_seg[E/W] = rows it receives);
+ *   recv_counts: int32 [E/W] slots routed to each of this rank's experts by
+ *     all ranks (the grouped GEMM's per-expert row counts). */
+ep_status ep_plan_export(const ep_plan *plan, int32_t *dst, int32_t *recv_seg, int32_t *recv_counts,
+                         ep_stream_t stream);
+/* Rows this rank receives (host; synchronises the stream). */
+ep_status ep_plan_recv_rows_host(const ep_plan *plan, int64_t *rows, ep_stream_t stream);
+/* The plan's device error word (synchronises): EP_OK or EP_ERR_CAPACITY. */
+ep_status ep_plan_check(const ep_plan *plan, ep_stream_t stream);
+
+typedef struct ep_peers ep_peers;
+
+/* Table of every rank's buffers as mapped in this process (host arrays of
+ * `world` device pointers, entry r for rank r, this rank's own included):
+ *   recv_x: receive buffers, [recv_rows, H] bf16 or e4m3, 16-byte aligned;
+ *   recv_scales: FP8 scale buffers, fp32 [recv_rows, H/128] row-major, or
+ *     NULL (BF16 dispatch only);
+ *   y: expert-output buffers, bf16 [recv_rows, H] in receive-row order, or
+ *     NULL (no combine).
+ * Each pointer is checked on the host (non-NULL, 16-byte aligned) and the
+ * tables are copied to device memory the object owns (ep_peers_free).  The
+ * buffers themselves stay the caller's. */
+ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_scales, void *const *y,
+                          size_t recv_rows, ep_peers **out);
+void ep_peers_free(ep_peers *peers);
+
+/* Dispatch across ranks: as ep_dispatch_ex, with row (d.y) of rank d.x's
+ * buffers as the destination of each slot (d from the plan), written with
+ * plain 16-byte stores through the peer mappings; scales row-major.  The
+ * caller orders these stores before the owners' reads with a collective. */
+ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const void *x, const float *x_scales,
+                           int hidden, int in_format, int out_format, int num_sms, ep_stream_t stream);
+
+/* Combine across ranks: as ep_combine_ex, reading each slot's expert-output
+ * row from its owner's y buffer through the peer mappings.  topk_weights
+ * NULL means every weight 1, which is the backward of ep_dispatch_peer (the
+ * pages: a dispatch's backward is a combine). */
+ep_status ep_combine_peer(const ep_plan *plan, const ep_peers *peers, const float *topk_weights, int hidden,
+                          void *combined_x, int num_sms, ep_stream_t stream);
+
+/* CUDA IPC for the peer table.  ep_ipc_export writes the 64-byte handle of
+ * the cudaMalloc allocation that holds `ptr` and ptr's offset in it (host
+ * outputs); another process on the same node opens it with ep_ipc_import
+ * (peer access enabled lazily) and closes it with ep_ipc_release(ptr,
+ * offset).  Allocations made through the virtual-memory API (e.g. an
+ * expandable-segments allocator) cannot be exported: EP_ERR_CUDA. */
+#define EP_IPC_HANDLE_BYTES 64
+ep_status ep_ipc_export(const void *ptr, void *handle, uint64_t *offset);
+ep_status ep_ipc_import(const void *handle, uint64_t offset, void **ptr);
+ep_status ep_ipc_release(void *ptr, uint64_t offset);
+
 #ifdef __cplusplus
 }
 #endif
