@@ -21,7 +21,8 @@
  *
  * On one GPU the expert-parallel ranks are virtual: rank r owns experts
  * [r*E/R, (r+1)*E/R) and the contiguous slice of receive rows of those
- * experts.  Nothing crosses devices.
+ * experts.  The calls at the end of this header run the same contract with
+ * the ranks as real GPUs, one process each.
  *
  * Notation: T tokens, H hidden size, k top-k slots per token, E experts,
  * R virtual ranks.  A slot is a pair (t, j), 0 <= j < k.
