@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-cpu-baseline] [--no-e2e] [--no-decode]
-                    [--no-backward] [--no-overlap]
+                    [--no-backward] [--no-overlap] [--no-ranks]
 
 A step is one pass of the whole path over one batch: ep_layout (2 kernels),
 ep_dispatch (FP8 e4m3 or BF16), ep_combine (BF16), all through the C ABI.
@@ -51,8 +51,8 @@ HBM_FALLBACK_GBS = 6650.0
 # kernel source it was taken on (stale -> reported as null).
 NCU_TRAFFIC = {
     # one "ncu --set full" capture of one launch each on the metric workload
-    ("group_limited", "combine"): {"sha": "5dba458197e1f277", "bytes": 940058880 + 71877120},
-    ("group_limited", "dispatch"): {"sha": "557118bc734ec7e1", "bytes": 117844992 + 427099136},
+    ("group_limited", "combine"): {"sha": "4fbe5c822556c1bf", "bytes": 940077312 + 72000512},
+    ("group_limited", "dispatch"): {"sha": "e29b25d97fe7e03a", "bytes": 117793792 + 426959104},
 }
 
 
@@ -68,6 +68,7 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-backward", action="store_true")
     p.add_argument("--no-overlap", action="store_true")
+    p.add_argument("--no-ranks", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
 
@@ -520,6 +521,10 @@ def run_ours(args, w):
     if not args.no_overlap:
         overlap = run_overlap(w, dev, ep, idx, x, tw, y, flush_l2)
 
+    ranks = None
+    if world == 1 and not args.no_ranks:
+        ranks = run_ranks_emulated(w, dev, ep, flush_l2)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed)
@@ -532,7 +537,7 @@ def run_ours(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "decode": decode, "backward": backward, "overlap": overlap,
+            "decode": decode, "backward": backward, "overlap": overlap, "ranks_emulated": ranks,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "wall_s": wall,
             "host_us_per_step": host_s * 1e6,
         }
@@ -671,6 +676,79 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
     return {"dispatch_backward": {"us": d_us, "bytes": d_bytes, "gbs": d_bytes / d_us / 1e3},
             "combine_backward": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3},
             "dispatch_topk": {"us": t_us, "bytes": t_bytes, "note": "latency-bound (~1.6 MB)"}}
+
+
+def run_ranks_emulated(w, dev, ep, flush_l2, worlds=(1, 8), steps: int = 10) -> dict:
+    """Expert parallelism across W ranks, every rank emulated on this GPU:
+    the workload split into W source batches of T/W tokens, each rank's plan,
+    then every rank's peer dispatch and peer combine (each rank's kernels in
+    turn on one stream, all buffers in this GPU's HBM).  W = 1 runs the whole
+    batch through the peer-addressed kernels (compare with the local ones:
+    the cost of the indirection); W = 8 gives the plan's latency at eight
+    ranks and eight back-to-back launches of T/8 tokens.  Not NVLink, which
+    needs GPUs."""
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        ts = []
+        for i in range(steps + 3):
+            flush_l2()
+            torch.cuda._sleep(GPU_LEAD_CYCLES)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if i >= 3:
+                ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ts) * 1e3
+
+    out = {"note": "all ranks emulated on one GPU: every store and load is local HBM, no NVLink"}
+    for world in worlds:
+        Tr = w.T // world
+        parts = [W.make_routing(w.scaled(T=Tr), seed=7000 + r) for r in range(world)] if world > 1 else \
+            [W.make_routing(w, seed=0)]
+        rows = ep.ep_peer_max_recv_rows(Tr * world, w.k, w.E, world)
+        rdt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
+        recv = [torch.empty(rows, w.H, dtype=rdt, device=dev) for _ in range(world)]
+        sc = [torch.empty(rows, w.H // 128, dtype=torch.float32, device=dev) for _ in range(world)] \
+            if w.fp8 else None
+        g = torch.Generator(device=dev).manual_seed(99)
+        ys = [torch.randn(rows, w.H, generator=g, device=dev).to(torch.bfloat16) for _ in range(world)]
+        peers = ep.Peers(world, recv, sc, ys, rows)
+        xs = [p[0].to(dev) for p in parts]
+        idxs = [p[1].to(dev) for p in parts]
+        tws = [p[2].to(dev) for p in parts]
+        lays = [ep.ep_layout(i, w.E, world) for i in idxs]
+        counts = torch.stack([l.num_tokens_per_expert for l in lays])
+        plans = [ep.ep_plan_create(l.handle, i, counts, r, world, rows)
+                 for r, (l, i) in enumerate(zip(lays, idxs))]
+        plan_us = timed(lambda: ep.ep_plan_create(lays[0].handle, idxs[0], counts, 0, world, rows).free())
+        d_us = timed(lambda: [ep.ep_dispatch_peer(plans[r], peers, xs[r], w.fp8) for r in range(world)])
+        c_us = timed(lambda: [ep.ep_combine_peer(plans[r], peers, tws[r], w.H) for r in range(world)])
+        if any(p.check() != ep.EP_OK for p in plans):
+            raise SystemExit("ranks_emulated: plan error")
+        V = sum(int((p[1] >= 0).sum()) for p in parts)
+        T = Tr * world
+        if w.fp8:
+            d_bytes = T * w.H * 2 + V * w.H + V * (w.H // 128) * 4 + T * w.k * 8
+        else:
+            d_bytes = T * w.H * 2 + V * w.H * 2 + T * w.k * 8
+        c_bytes = V * w.H * 2 + T * w.k * 12 + T * w.H * 2
+        out["world_%d" % world] = {
+            "tokens_per_rank": Tr, "plan_us": plan_us,
+            "dispatch": {"us": d_us, "bytes": d_bytes, "gbs": d_bytes / d_us / 1e3},
+            "combine": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3},
+            "recv_rows_per_rank": [p.recv_rows_host() for p in plans]}
+        for p in plans:
+            p.free()
+        for l in lays:
+            l.handle.free()
+        peers.free()
+        del recv, sc, ys
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_overlap(w, dev, ep, idx_dev, x_dev, tw_dev, y_dev, flush_l2, reps: int = 10) -> dict:
