@@ -93,11 +93,27 @@ def combine(RL: RankedLayout, y_list, w_list):
     """y_list[r]: bf16 [>= recv_rows(r), H] expert outputs on rank r, rows in
     its receive order; w_list[s]: float32 [T_s, k].  Returns the combined
     uint16 [T_s, H] of every source rank."""
+    w = np.concatenate([np.asarray(a, np.float32) for a in w_list])
+    out = oracle.combine(_concat_y(RL, y_list), w, RL.L.pos)
+    return [out[b:b + T] for b, T in zip(RL.token_base, RL.T)]
+
+
+def _concat_y(RL: RankedLayout, y_list):
     H = oracle._u16(y_list[0]).shape[1]
     y = np.zeros((max(RL.L.n_rows, 1), H), np.uint16)
     for r in range(RL.W):
         n = RL.recv_rows(r)
         y[RL.L.rank_off[r]:RL.L.rank_off[r] + n] = oracle._u16(y_list[r])[:n]
+    return y[:RL.L.n_rows]
+
+
+def combine_backward(RL: RankedLayout, grad_out_list, y_list, w_list):
+    """The backward of `combine` across ranks (the pages: a combine's backward
+    is a dispatch).  grad_out_list[s]: bf16 [T_s, H]; y_list[r]: the owner's
+    expert outputs.  Returns (grad_y per owner rank, uint16 [recv_rows(r), H],
+    rows no slot fills are 0; grad_w per source rank, float64 [T_s, k])."""
+    g = _concat_u16(grad_out_list)
     w = np.concatenate([np.asarray(a, np.float32) for a in w_list])
-    out = oracle.combine(y[:RL.L.n_rows], w, RL.L.pos)
-    return [out[b:b + T] for b, T in zip(RL.token_base, RL.T)]
+    gy, gw = oracle.combine_backward(g, _concat_y(RL, y_list), w, RL.L.pos)
+    return ([gy[RL.L.rank_off[r]:RL.L.rank_off[r + 1]] for r in range(RL.W)],
+            [gw[b:b + T] for b, T in zip(RL.token_base, RL.T)])

@@ -126,3 +126,29 @@ def test_padded_capacity_in_concatenated_token_order():
     assert RL.recv_counts(0).tolist() == [4] and RL.recv_counts(1).tolist() == [1]
     st, _ = MR.layout([idx0, idx1], 2, 2, 1, 3, check=False)
     assert st == oracle.OR_ERR_CAPACITY
+
+
+def test_combine_backward_by_enumeration():
+    """grad_y of the slot (s, t, j) sits on its owner at the row the brute-force
+    enumeration gives it and equals bf16(fp32(w * g)); grad_w[s][t][j] is the
+    dot product of g with that row of the owner's y (exact in binary64)."""
+    rng = np.random.default_rng(21)
+    W_, E, k, H = 3, 6, 2, 16
+    idx_list = [random_ids(rng, T, k, E, unused=0.2) for T in (4, 0, 5)]
+    _, RL = MR.layout(idx_list, E, W_)
+    g_list = [torch.from_numpy(rng.standard_normal((i.shape[0], H))).to(torch.bfloat16) for i in idx_list]
+    w_list = [rng.random(i.shape).astype(np.float32) for i in idx_list]
+    y_list = [torch.from_numpy(rng.standard_normal((max(RL.recv_rows(r), 1), H))).to(torch.bfloat16)
+              for r in range(W_)]
+    gy, gw = MR.combine_backward(RL, g_list, y_list, w_list)
+    want = brute_rows(idx_list, E, W_, 1)
+    for r in range(W_):
+        assert gy[r].shape[0] == RL.recv_rows(r)
+        for row, who in enumerate(want[r]):
+            s, t, j = who
+            prod = torch.tensor(float(w_list[s][t, j]), dtype=torch.float32) * g_list[s][t].float()
+            assert (gy[r][row] == oracle._u16(prod.to(torch.bfloat16))).all()
+            dot = float((g_list[s][t].double() * y_list[r][row].double()).sum())
+            assert abs(gw[s][t, j] - dot) <= 1e-12 * (1 + abs(dot))
+    for s, idx in enumerate(idx_list):
+        assert (gw[s][idx < 0] == 0).all()
