@@ -20,6 +20,11 @@
 // (16 loads in flight per thread; 128 threads x 4 blocks per SM measured best).
 // The result is deterministic run to run; its distance from the exact dot
 // product is bounded by (#additions on the longest path) x 2^-24 x sum|g*y|.
+// Threads j < k first resolve each slot's y row and grad_y row to pointers:
+// row pos[t][j] of the local buffers, or, when the ranks are real GPUs
+// (PEER), row d.y of rank d.x's buffers (d = dst[t][j] of the plan) through
+// the peer table: the weighted scatter then stores straight into the owner's
+// gradient buffer and the dot products read the owner's y.
 #include <cuda_bf16.h>
 
 #include "ep_internal.cuh"
@@ -55,17 +60,36 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 constexpr int kBwdBatch = EP_BWD_BATCH;  // slots whose y rows are loaded before any is used
 constexpr int kBwdMaxThreads = EP_BWD_MAX_THREADS;
 
-template <int KMAX, bool NEED_W>
+template <int KMAX, bool NEED_W, bool PEER>
 __global__ void __launch_bounds__(kBwdMaxThreads, EP_BWD_MIN_BLOCKS) combine_bwd_kernel(CombineBwdArgs a) {
-    __shared__ int32_t p_s[KMAX];
+    __shared__ const uint8_t *y_s[KMAX];
+    __shared__ uint8_t *gy_s[KMAX];
     __shared__ float w_s[KMAX];
     __shared__ float red_s[kBwdMaxThreads / 32][KMAX];
     pdl_wait_then_trigger();
     const int t = blockIdx.x;
     const int tid = threadIdx.x;
+    const size_t row_bytes = (size_t)a.H * 2;
     if (tid < a.k) {
-        p_s[tid] = __ldg(a.pos + (int64_t)t * a.k + tid);
-        w_s[tid] = __ldg(a.w + (int64_t)t * a.k + tid);
+        const int64_t s = (int64_t)t * a.k + tid;
+        const uint8_t *yr = nullptr;
+        uint8_t *gr = nullptr;
+        if (PEER) {
+            const int2 d = __ldg(a.dst + s);
+            if (d.x >= 0) {
+                gr = a.peer_grad_y[d.x] + (size_t)d.y * row_bytes;
+                if (NEED_W) yr = a.peer_y[d.x] + (size_t)d.y * row_bytes;
+            }
+        } else {
+            const int p = __ldg(a.pos + s);
+            if (p >= 0) {
+                gr = a.grad_y + (size_t)p * row_bytes;
+                if (NEED_W) yr = a.y + (size_t)p * row_bytes;
+            }
+        }
+        y_s[tid] = yr;
+        gy_s[tid] = gr;
+        w_s[tid] = __ldg(a.w + s);
     }
     __syncthreads();
 
@@ -73,10 +97,7 @@ __global__ void __launch_bounds__(kBwdMaxThreads, EP_BWD_MIN_BLOCKS) combine_bwd
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) part[j] = 0.0f;
 
-    const size_t row_bytes = (size_t)a.H * 2;
     const uint8_t *__restrict__ g_row = a.grad_out + (size_t)t * row_bytes;
-    const uint8_t *__restrict__ ybase = a.y;
-    uint8_t *__restrict__ gybase = a.grad_y;
     for (int c = tid; c * 16 < a.H; c += blockDim.x) {
         const size_t off = (size_t)c * 32;      // 16 channels = 32 bytes
         const bool full = c * 16 + 16 <= a.H;  // H % 16 == 8: the last group has 8 channels
@@ -97,21 +118,20 @@ __global__ void __launch_bounds__(kBwdMaxThreads, EP_BWD_MIN_BLOCKS) combine_bwd
 #pragma unroll
                 for (int jj = 0; jj < kBwdBatch; ++jj) {
                     const int j = j0 + jj;
-                    const int p = (j < a.k) ? p_s[j] : -1;
+                    const uint8_t *yr = (j < a.k) ? y_s[j] : nullptr;
                     yv[jj][0] = make_uint4(0u, 0u, 0u, 0u);
                     yv[jj][1] = yv[jj][0];
-                    if (p >= 0) {
-                        const uint8_t *y_row = ybase + (size_t)p * row_bytes + off;
-                        yv[jj][0] = ld_nc_v4(y_row);
-                        if (full) yv[jj][1] = ld_nc_v4(y_row + 16);
+                    if (yr != nullptr) {
+                        yv[jj][0] = ld_nc_v4(yr + off);
+                        if (full) yv[jj][1] = ld_nc_v4(yr + off + 16);
                     }
                 }
             }
 #pragma unroll
             for (int jj = 0; jj < kBwdBatch; ++jj) {
                 const int j = j0 + jj;
-                const int p = (j < a.k) ? p_s[j] : -1;
-                if (p < 0) continue;
+                uint8_t *gr = (j < a.k) ? gy_s[j] : nullptr;
+                if (gr == nullptr) continue;
                 if (NEED_W) {
                     float y[16];
                     unpack8(yv[jj][0], y);
@@ -131,7 +151,7 @@ __global__ void __launch_bounds__(kBwdMaxThreads, EP_BWD_MIN_BLOCKS) combine_bwd
                 o1.y = pack_bf16x2(__fmul_rn(wj, g[10]), __fmul_rn(wj, g[11]));
                 o1.z = pack_bf16x2(__fmul_rn(wj, g[12]), __fmul_rn(wj, g[13]));
                 o1.w = pack_bf16x2(__fmul_rn(wj, g[14]), __fmul_rn(wj, g[15]));
-                uint8_t *dst = gybase + (size_t)p * row_bytes + off;
+                uint8_t *dst = gr + off;
                 *reinterpret_cast<uint4 *>(dst) = o0;
                 if (full) *reinterpret_cast<uint4 *>(dst + 16) = o1;
             }
@@ -157,23 +177,32 @@ __global__ void __launch_bounds__(kBwdMaxThreads, EP_BWD_MIN_BLOCKS) combine_bwd
     if (tid < a.k) {
         float s = 0.0f;
         for (int w = 0; w < nwarps; ++w) s += red_s[w][tid];
-        a.grad_w[(int64_t)t * a.k + tid] = (p_s[tid] >= 0) ? s : 0.0f;
+        a.grad_w[(int64_t)t * a.k + tid] = (gy_s[tid] != nullptr) ? s : 0.0f;
     }
 }
 
-}  // namespace
-
-cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s) {
+template <bool PEER>
+cudaError_t launch_combine_backward_impl(const CombineBwdArgs &a, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     // One thread per 16 channels, at most kBwdMaxThreads; threads loop over the rest.
     const int groups = (a.H + 15) / 16;
     const int threads = groups >= kBwdMaxThreads ? kBwdMaxThreads : ((groups + 31) / 32) * 32;
     const bool need_w = a.grad_w != nullptr;
     if (a.k <= 8)
-        return need_w ? launch_kernel(combine_bwd_kernel<8, true>, a.T, threads, 0, s, a)
-                      : launch_kernel(combine_bwd_kernel<8, false>, a.T, threads, 0, s, a);
-    return need_w ? launch_kernel(combine_bwd_kernel<kMaxTopk, true>, a.T, threads, 0, s, a)
-                  : launch_kernel(combine_bwd_kernel<kMaxTopk, false>, a.T, threads, 0, s, a);
+        return need_w ? launch_kernel(combine_bwd_kernel<8, true, PEER>, a.T, threads, 0, s, a)
+                      : launch_kernel(combine_bwd_kernel<8, false, PEER>, a.T, threads, 0, s, a);
+    return need_w ? launch_kernel(combine_bwd_kernel<kMaxTopk, true, PEER>, a.T, threads, 0, s, a)
+                  : launch_kernel(combine_bwd_kernel<kMaxTopk, false, PEER>, a.T, threads, 0, s, a);
+}
+
+}  // namespace
+
+cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s) {
+    return launch_combine_backward_impl<false>(a, s);
+}
+
+cudaError_t launch_combine_backward_peer(const CombineBwdArgs &a, cudaStream_t s) {
+    return launch_combine_backward_impl<true>(a, s);
 }
 
 }  // namespace ep

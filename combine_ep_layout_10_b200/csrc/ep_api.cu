@@ -591,12 +591,13 @@ struct ep_peers {
     uint8_t *const *recv_x;      // [world]
     float *const *recv_scales;   // [world] or nullptr
     const uint8_t *const *y;     // [world] or nullptr
+    uint8_t *const *grad_y;      // [world] or nullptr
 };
 
 extern "C" {
 
 ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_scales, void *const *y,
-                          size_t recv_rows, ep_peers **out) {
+                          void *const *grad_y, size_t recv_rows, ep_peers **out) {
     if (out == nullptr) return EP_ERR_INVALID_ARG;
     *out = nullptr;
     if (world < 1 || recv_x == nullptr) return EP_ERR_INVALID_ARG;
@@ -604,6 +605,7 @@ ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_sca
         if (recv_x[r] == nullptr || !aligned(recv_x[r], 16)) return EP_ERR_INVALID_ARG;
         if (recv_scales && (recv_scales[r] == nullptr || !aligned(recv_scales[r], 16))) return EP_ERR_INVALID_ARG;
         if (y && (y[r] == nullptr || !aligned(y[r], 16))) return EP_ERR_INVALID_ARG;
+        if (grad_y && (grad_y[r] == nullptr || !aligned(grad_y[r], 16))) return EP_ERR_INVALID_ARG;
     }
     int dev;
     DeviceInfo info;
@@ -615,7 +617,7 @@ ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_sca
     p->device = dev;
     p->recv_rows = recv_rows;
     const size_t n = (size_t)world;
-    uintptr_t *host = static_cast<uintptr_t *>(std::malloc(3 * n * sizeof(uintptr_t)));
+    uintptr_t *host = static_cast<uintptr_t *>(std::malloc(4 * n * sizeof(uintptr_t)));
     if (host == nullptr) {
         delete p;
         return EP_ERR_OOM;
@@ -624,9 +626,10 @@ ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_sca
         host[r] = reinterpret_cast<uintptr_t>(recv_x[r]);
         host[n + r] = recv_scales ? reinterpret_cast<uintptr_t>(recv_scales[r]) : 0;
         host[2 * n + r] = y ? reinterpret_cast<uintptr_t>(y[r]) : 0;
+        host[3 * n + r] = grad_y ? reinterpret_cast<uintptr_t>(grad_y[r]) : 0;
     }
-    cudaError_t e = cudaMalloc(&p->block, 3 * n * sizeof(uintptr_t));
-    if (e == cudaSuccess) e = cudaMemcpy(p->block, host, 3 * n * sizeof(uintptr_t), cudaMemcpyHostToDevice);
+    cudaError_t e = cudaMalloc(&p->block, 4 * n * sizeof(uintptr_t));
+    if (e == cudaSuccess) e = cudaMemcpy(p->block, host, 4 * n * sizeof(uintptr_t), cudaMemcpyHostToDevice);
     std::free(host);
     if (e != cudaSuccess) {
         if (p->block) cudaFree(p->block);
@@ -637,6 +640,7 @@ ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_sca
     p->recv_x = reinterpret_cast<uint8_t *const *>(tab);
     p->recv_scales = recv_scales ? reinterpret_cast<float *const *>(tab + n) : nullptr;
     p->y = y ? reinterpret_cast<const uint8_t *const *>(tab + 2 * n) : nullptr;
+    p->grad_y = grad_y ? reinterpret_cast<uint8_t *const *>(tab + 3 * n) : nullptr;
     *out = p;
     return EP_OK;
 }
@@ -714,6 +718,33 @@ ep_status ep_combine_peer(const ep_plan *plan, const ep_peers *peers, const floa
     if ((int64_t)plan->T * a.blocks_per_token >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.num_sms = num_sms;
     return cuda_status(launch_combine_peer(a, stream));
+}
+
+ep_status ep_combine_backward_peer(const ep_plan *plan, const ep_peers *peers, const void *grad_out,
+                                   const float *topk_w, int H, float *grad_w, ep_stream_t stream) {
+    if (plan == nullptr || peers == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (peers->world != plan->world || peers->grad_y == nullptr || peers->recv_rows < (size_t)plan->recv_rows)
+        return EP_ERR_INVALID_ARG;
+    if (grad_w != nullptr && peers->y == nullptr) return EP_ERR_INVALID_ARG;
+    if (plan->T > 0) {
+        if (grad_out == nullptr || topk_w == nullptr) return EP_ERR_INVALID_ARG;
+        if (!aligned(grad_out, 16) || !aligned(topk_w, 4)) return EP_ERR_INVALID_ARG;
+        if (grad_w != nullptr && !aligned(grad_w, 4)) return EP_ERR_INVALID_ARG;
+    }
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != plan->device || dev != peers->device) return EP_ERR_INVALID_ARG;
+    CombineBwdArgs a{};
+    a.grad_out = static_cast<const uint8_t *>(grad_out);
+    a.w = topk_w;
+    a.grad_w = grad_w;
+    a.dst = plan->dst;
+    a.peer_y = peers->y;
+    a.peer_grad_y = peers->grad_y;
+    a.T = plan->T; a.k = plan->k; a.H = H;
+    return cuda_status(launch_combine_backward_peer(a, stream));
 }
 
 ep_status ep_ipc_export(const void *ptr, void *handle, uint64_t *offset) {

@@ -223,6 +223,10 @@ struct CombineBwdArgs {
     uint8_t *grad_y;         // bf16 [rows, H]
     float *grad_w;           // [T, k] or nullptr
     int T, k, H;
+    // Multi-rank (peer) addressing, used instead of pos / y / grad_y:
+    const int2 *dst;                 // [T, k] (rank, row) of each slot, rank -1 if none
+    const uint8_t *const *peer_y;    // [world] every rank's expert outputs
+    uint8_t *const *peer_grad_y;     // [world] every rank's grad_y buffer
 };
 
 struct RecvTopkArgs {
@@ -295,6 +299,7 @@ cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
 // Peer-addressed variants of dispatch and combine (DispatchArgs::dst, CombineArgs::src).
 cudaError_t launch_dispatch_peer(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine_peer(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_combine_backward_peer(const CombineBwdArgs &a, cudaStream_t s);
 
 // Per-device facts, cached.
 struct DeviceInfo {

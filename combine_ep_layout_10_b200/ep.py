@@ -40,6 +40,7 @@ ABI_SYMBOLS = (
     "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk",
     "ep_peer_max_recv_rows", "ep_plan_create", "ep_plan_free", "ep_plan_export", "ep_plan_recv_rows_host",
     "ep_plan_check", "ep_peers_create", "ep_peers_free", "ep_dispatch_peer", "ep_combine_peer",
+    "ep_combine_backward_peer",
     "ep_ipc_export", "ep_ipc_import", "ep_ipc_release",
 )
 
@@ -120,7 +121,7 @@ def lib() -> ctypes.CDLL:
         L.ep_plan_recv_rows_host.restype = I
         L.ep_plan_check.argtypes = [P, P]
         L.ep_plan_check.restype = I
-        L.ep_peers_create.argtypes = [I, P, P, P, S, ctypes.POINTER(P)]
+        L.ep_peers_create.argtypes = [I, P, P, P, P, S, ctypes.POINTER(P)]
         L.ep_peers_create.restype = I
         L.ep_peers_free.argtypes = [P]
         L.ep_peers_free.restype = None
@@ -128,6 +129,8 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_peer.restype = I
         L.ep_combine_peer.argtypes = [P, P, P, I, P, I, P]
         L.ep_combine_peer.restype = I
+        L.ep_combine_backward_peer.argtypes = [P, P, P, P, I, P, P]
+        L.ep_combine_backward_peer.restype = I
         L.ep_ipc_export.argtypes = [P, P, ctypes.POINTER(U64)]
         L.ep_ipc_export.restype = I
         L.ep_ipc_import.argtypes = [P, U64, ctypes.POINTER(P)]
@@ -523,11 +526,13 @@ def _ptr_array(ptrs):
 class Peers:
     """Owner of an ep_peers*: every rank's buffers as addressed from this process."""
 
-    def __init__(self, world: int, recv_x, recv_scales, y, recv_rows: int):
+    def __init__(self, world: int, recv_x, recv_scales, y, recv_rows: int, grad_y=None):
         out = ctypes.c_void_p()
         st = lib().ep_peers_create(world, _ptr_array(recv_x),
                                    _ptr_array(recv_scales) if recv_scales is not None else None,
-                                   _ptr_array(y) if y is not None else None, recv_rows, ctypes.byref(out))
+                                   _ptr_array(y) if y is not None else None,
+                                   _ptr_array(grad_y) if grad_y is not None else None, recv_rows,
+                                   ctypes.byref(out))
         _check(st, "ep_peers_create")
         self._ptr = out
         self.world = world
@@ -579,6 +584,26 @@ def ep_combine_peer(plan: Plan, peers: Peers, topk_weights: Optional[torch.Tenso
                                num_sms, _stream(stream))
     _check(st, "ep_combine_peer")
     return out
+
+
+def ep_combine_backward_peer(plan: Plan, peers: Peers, grad_out: torch.Tensor, topk_weights: torch.Tensor,
+                             want_grad_weights: bool = True, grad_weights: Optional[torch.Tensor] = None,
+                             stream=None) -> Optional[torch.Tensor]:
+    """Stores each local slot's gradient row into its owner's grad_y buffer;
+    returns grad_weights [T, k] fp32 (dot products with the owners' y rows) or None."""
+    T, H = grad_out.shape
+    if want_grad_weights and grad_weights is None:
+        grad_weights = torch.empty(T, plan.num_topk, dtype=torch.float32, device=grad_out.device)
+    if not want_grad_weights:
+        grad_weights = None
+    st = lib().ep_combine_backward_peer(plan.ptr, peers.ptr,
+                                        _dev_ptr(grad_out, torch.bfloat16, "grad_out", (plan.num_tokens, H)),
+                                        _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                                 (plan.num_tokens, plan.num_topk)),
+                                        H, _dev_ptr(grad_weights, torch.float32, "grad_weights",
+                                                    (plan.num_tokens, plan.num_topk)), _stream(stream))
+    _check(st, "ep_combine_backward_peer")
+    return grad_weights
 
 
 def ipc_export(t: torch.Tensor):

@@ -11,6 +11,10 @@ collectives that order one rank's stores before another rank's reads:
 
     dispatch:  layout -> all-gather counts -> plan -> peer stores -> barrier
     combine:   barrier (every y written) -> peer loads
+    backward:  combine_backward: barrier -> peer stores of grad_y (+ grad_w
+               from the owners' y) -> barrier; dispatch_backward: barrier
+               (every owner wrote its receive-row gradients into its y
+               buffer) -> peer loads with unit weights
 
 The next dispatch's all-gather (or, with a cached plan, its barrier) orders
 its stores after every rank's reads of the previous step.  No kernel waits
@@ -51,13 +55,14 @@ class EpGroup:
                                   device=dev)
         self.recv_scales = torch.empty(recv_rows, hidden // 128, dtype=torch.float32, device=dev) if fp8 else None
         self.y = torch.empty(recv_rows, hidden, dtype=torch.bfloat16, device=dev)
-        mine = [self.recv_x, self.recv_scales, self.y]
+        self.grad_y = torch.empty(recv_rows, hidden, dtype=torch.bfloat16, device=dev)
+        mine = [self.recv_x, self.recv_scales, self.y, self.grad_y]
         handles = [ep.ipc_export(t) if t is not None else None for t in mine]
         torch.cuda.synchronize(dev)
         everyone = [None] * self.world
         dist.all_gather_object(everyone, handles, group=group)
         self._imported = []   # (address, offset) to release
-        tables = [[], [], []]
+        tables = [[], [], [], []]
         for r in range(self.world):
             for i, t in enumerate(mine):
                 if t is None:
@@ -69,7 +74,8 @@ class EpGroup:
                     addr = ep.ipc_import(blob, off)
                     self._imported.append((addr, off))
                     tables[i].append(addr)
-        self.peers = ep.Peers(self.world, tables[0], tables[1] if fp8 else None, tables[2], recv_rows)
+        self.peers = ep.Peers(self.world, tables[0], tables[1] if fp8 else None, tables[2], recv_rows,
+                              grad_y=tables[3])
 
     # -- collectives -------------------------------------------------------
 
@@ -122,6 +128,24 @@ class EpGroup:
         owners' `y` buffers (the caller has written its own `y` rows)."""
         self._barrier()       # every rank's y is written
         return ep.ep_combine_peer(plan, self.peers, topk_weights, self.H, num_sms=num_sms)
+
+    def combine_backward(self, plan: ep.Plan, grad_out: torch.Tensor, topk_weights: torch.Tensor,
+                         want_grad_weights: bool = True) -> Optional[torch.Tensor]:
+        """Backward of `combine`: every local slot's gradient row
+        bf16(w * grad_out[t]) lands in its owner's `grad_y` buffer; returns
+        grad_weights [T, k] (dot products with the owners' y rows) or None."""
+        self._barrier()       # owners have finished with the previous grad_y
+        gw = ep.ep_combine_backward_peer(plan, self.peers, grad_out, topk_weights, want_grad_weights)
+        self._barrier()       # every rank's gradient rows are stored
+        return gw
+
+    def dispatch_backward(self, plan: ep.Plan) -> torch.Tensor:
+        """Backward of `dispatch`: each local token's sum of its receive-row
+        gradients, read from the owners' `y` buffers, into which every rank's
+        expert backward has written its receive-row gradients (y is no longer
+        needed once combine_backward has run)."""
+        self._barrier()       # every owner's receive-row gradients are written
+        return ep.ep_combine_peer(plan, self.peers, None, self.H)
 
     def close(self) -> None:
         """Release the peer mappings (after a final barrier, so no rank still

@@ -398,12 +398,14 @@ typedef struct ep_peers ep_peers;
  *   recv_scales: FP8 scale buffers, fp32 [recv_rows, H/128] row-major, or
  *     NULL (BF16 dispatch only);
  *   y: expert-output buffers, bf16 [recv_rows, H] in receive-row order, or
- *     NULL (no combine).
+ *     NULL (no combine);
+ *   grad_y: buffers the combine backward writes the expert-output gradients
+ *     into, bf16 [recv_rows, H] in receive-row order, or NULL.
  * Each pointer is checked on the host (non-NULL, 16-byte aligned) and the
  * tables are copied to device memory the object owns (ep_peers_free).  The
  * buffers themselves stay the caller's. */
 ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_scales, void *const *y,
-                          size_t recv_rows, ep_peers **out);
+                          void *const *grad_y, size_t recv_rows, ep_peers **out);
 void ep_peers_free(ep_peers *peers);
 
 /* Dispatch across ranks: as ep_dispatch_ex, with row (d.y) of rank d.x's
@@ -419,6 +421,19 @@ ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const voi
  * pages: a dispatch's backward is a combine). */
 ep_status ep_combine_peer(const ep_plan *plan, const ep_peers *peers, const float *topk_weights, int hidden,
                           void *combined_x, int num_sms, ep_stream_t stream);
+
+/* Combine backward across ranks: as ep_combine_backward, with each slot's
+ * gradient row bf16_rn(fp32_rn(w[t][j] * grad_out[t])) stored into its
+ * owner's grad_y buffer and grad_w[t][j] = <grad_out[t], y row> read from
+ * the owner's y buffer (the pages: a combine's backward is a dispatch).
+ *   grad_out: device bf16 [T, H]; topk_weights: device fp32 [T, k];
+ *   grad_w: device fp32 [T, k], or NULL to skip the dot products (then the
+ *     peers' y table may be NULL).  Needs the peers' grad_y table.
+ * Rows no slot fills are not written.  The caller orders the stores before
+ * the owners' reads with a collective, as for ep_dispatch_peer. */
+ep_status ep_combine_backward_peer(const ep_plan *plan, const ep_peers *peers, const void *grad_out,
+                                   const float *topk_weights, int hidden, float *grad_w,
+                                   ep_stream_t stream);
 
 /* CUDA IPC for the peer table.  ep_ipc_export writes the 64-byte handle of
  * the cudaMalloc allocation that holds `ptr` and ptr's offset in it (host

@@ -62,7 +62,8 @@ class Emulated:
         self.scales = [torch.full((rows, H // 128), -1.0, dtype=torch.float32, device=DEV) for _ in range(self.W)] \
             if fp8 else None
         self.y = [torch.zeros(rows, H, dtype=torch.bfloat16, device=DEV) for _ in range(self.W)]
-        self.peers = ep.Peers(self.W, self.recv, self.scales, self.y, rows)
+        self.grad_y = [torch.full((rows, H), SENTINEL, dtype=torch.int16, device=DEV) for _ in range(self.W)]
+        self.peers = ep.Peers(self.W, self.recv, self.scales, self.y, rows, grad_y=self.grad_y)
         self.idx_dev = [i.to(DEV) for i in idx_list]
         self.layouts = [ep.ep_layout(i, E, self.W) for i in self.idx_dev]
         counts = torch.stack([l.num_tokens_per_expert for l in self.layouts])  # the all-gather
@@ -215,3 +216,57 @@ def test_plan_argument_errors():
     bad = torch.empty(64 * base.H + 8, dtype=torch.int16, device=DEV)[1:]
     with pytest.raises(ep.EpError):
         ep.Peers(2, [bad, bad], None, None, 64)  # misaligned buffer
+
+
+@pytest.mark.parametrize("name,Ts,align,H", [("prefill", [64, 30, 0, 100], 1, None),
+                                             ("group_limited", [300, 212], 8, None),
+                                             ("tiny", [64, 64], 4, 1000)])
+def test_peer_combine_backward(name, Ts, align, H):
+    """grad_y rows land bit-exactly on their owners; grad_w equals the local
+    kernel's on the concatenated layout bit for bit (the same per-token
+    reduction order) and the oracle within the derived bound."""
+    import math
+    base, idx_list, _, w_list = routing(name, Ts, unused=True, H=H)
+    Wr = len(Ts)
+    em = Emulated(base.E, base.k, base.H, idx_list, False, align)
+    _, RL = MR.layout(idx_list, base.E, Wr, align)
+    ys = []
+    for r in range(Wr):
+        y = W.make_expert_out(em.recv_rows, base.H, seed=500 + r)
+        em.y[r].copy_(y.to(DEV))
+        ys.append(y)
+    gos = [W.make_x(base.scaled(T=T), 600 + r) for r, T in enumerate(Ts)]
+    gws = [ep.ep_combine_backward_peer(em.plans[r], em.peers, gos[r].to(DEV), w_list[r].to(DEV))
+           for r in range(Wr)]
+    torch.cuda.synchronize()
+    want_gy, want_gw = MR.combine_backward(RL, gos, ys, w_list)
+    for r in range(Wr):
+        n = RL.recv_rows(r)
+        f = filled_rows(RL, r)
+        got = em.grad_y[r][:n].cpu().numpy().view(np.uint16)
+        assert (got[f] == want_gy[r][f]).all()
+        assert (em.grad_y[r][:n].cpu().numpy()[~f] == SENTINEL).all()
+    # the local kernel on the concatenated batch
+    idx_cat = torch.cat(idx_list)
+    res = ep.ep_layout(idx_cat.to(DEV), base.E, Wr, align)
+    y_cat = torch.zeros(res.handle.num_recv_rows, base.H, dtype=torch.bfloat16)
+    for r in range(Wr):
+        n = RL.recv_rows(r)
+        y_cat[RL.L.rank_off[r]:RL.L.rank_off[r] + n] = ys[r][:n]
+    _, gw_cat = ep.ep_combine_backward(res.handle, torch.cat(gos).to(DEV), torch.cat(w_list).to(DEV),
+                                       y=y_cat.to(DEV))
+    gw_cat = gw_cat.cpu()
+    for r in range(Wr):
+        b, T = RL.token_base[r], RL.T[r]
+        assert torch.equal(gws[r].cpu(), gw_cat[b:b + T])
+        g64 = gos[r].double().numpy()
+        bound = (16 * math.ceil(base.H / 2048) + 37) * 2.0 ** -24
+        d = RL.destinations(r)
+        for t in range(T):
+            for j in range(base.k):
+                if d[t, j, 0] < 0:
+                    assert gws[r][t, j].item() == 0.0
+                    continue
+                yrow = ys[d[t, j, 0]][d[t, j, 1]].double().numpy()
+                lim = bound * np.abs(g64[t] * yrow).sum() + 1e-30
+                assert abs(float(gws[r][t, j]) - want_gw[r][t, j]) <= lim

@@ -77,6 +77,22 @@ def _worker(rank, world, port, q):
         g.dispatch(x2[rank].cuda(), plan=plan)
         torch.cuda.synchronize()
         result["cached"] = check_recv(x2)
+        # backward: combine's (gradient rows to the owners), then dispatch's
+        gos = [W.make_x(base.scaled(T=T), 2000 + r) for r, T in enumerate(TOKENS)]
+        gw = g.combine_backward(plan, gos[rank].cuda(), w_list[rank].cuda())
+        torch.cuda.synchronize()
+        want_gy, want_gw = MR.combine_backward(RL, gos, ys, w_list)
+        got_gy = g.grad_y[:n].view(torch.int16).cpu().numpy().view(np.uint16)
+        scale = np.abs(gos[rank].double().numpy()).sum(1, keepdims=True) * 8.0
+        result["combine_bwd"] = bool((got_gy[filled] == want_gy[rank][filled]).all()
+                                     and (np.abs(gw.cpu().numpy() - want_gw[rank]) <= 1e-4 * scale).all())
+        grs = [W.make_expert_out(recv_rows, H, seed=3000 + r) for r in range(world)]
+        g.y.copy_(grs[rank].cuda())     # this rank's receive-row gradients
+        gx = g.dispatch_backward(plan)
+        torch.cuda.synchronize()
+        ones = [np.ones(i.shape, np.float32) for i in idx_list]
+        want_gx = MR.combine(RL, grs, ones)[rank]
+        result["dispatch_bwd"] = bool((gx.view(torch.int16).cpu().numpy().view(np.uint16) == want_gx).all())
         g.close()
         plan.free()
     except Exception as e:  # reported to the parent, which fails the test
@@ -110,3 +126,4 @@ def test_two_processes_share_buffers_over_ipc():
     for r in sorted(results, key=lambda d: d["rank"]):
         assert r["error"] is None, r
         assert r["dispatch"] and r["rows"] and r["combine"] and r["cached"], r
+        assert r["combine_bwd"] and r["dispatch_bwd"], r
