@@ -813,56 +813,81 @@ def run_overlap(w, dev, ep, idx_dev, x_dev, tw_dev, y_dev, flush_l2, reps: int =
 
 def run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y_dev, nbytes, world):
     """Same step through the public API from pinned host buffers: H2D of x,
-    topk_idx, topk_w and the expert outputs y, the three calls, D2H of out."""
+    topk_idx, topk_w and the expert outputs y, the three calls, D2H of out --
+    every step's copies inside the timed region.  Steps are pipelined two
+    deep, as a serving loop would run them: step n+1's uploads (one copy
+    stream) overlap step n's kernels (the compute stream) and step n-1's
+    readback (a second copy stream, the other PCIe direction); events order
+    each buffer set's reuse."""
     T, H, E, R = w.T, w.H, w.E, w.R
     xh = x_cpu.pin_memory()
     ih = idx_cpu.pin_memory()
     th = tw_cpu.pin_memory()
     yh = y_dev.cpu().pin_memory()
-    oh = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(xh, device=dev)
-    idd = torch.empty_like(ih, device=dev)
-    twd = torch.empty_like(th, device=dev)
-    yd = torch.empty_like(yh, device=dev)
+    ohs = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     rdt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
-    rows = yd.shape[0]
-    recv = torch.empty(rows, H, dtype=rdt, device=dev)
-    scales = torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if w.fp8 else None
-    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    rows = yh.shape[0]
+    sets = []
+    for _ in range(2):
+        sets.append({"x": torch.empty_like(xh, device=dev), "idx": torch.empty_like(ih, device=dev),
+                     "tw": torch.empty_like(th, device=dev), "y": torch.empty_like(yh, device=dev),
+                     "recv": torch.empty(rows, H, dtype=rdt, device=dev),
+                     "scales": torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if w.fp8 else None,
+                     "out": torch.empty(T, H, dtype=torch.bfloat16, device=dev)})
     h2d = sum(t.numel() * t.element_size() for t in (xh, ih, th, yh))
-    d2h = oh.numel() * oh.element_size()
-    stream = torch.cuda.current_stream()
+    d2h = ohs[0].numel() * ohs[0].element_size()
+    comp = torch.cuda.current_stream()
+    cin = torch.cuda.Stream(device=dev)
+    cout = torch.cuda.Stream(device=dev)
 
-    def step():
-        xd.copy_(xh, non_blocking=True)
-        idd.copy_(ih, non_blocking=True)
-        twd.copy_(th, non_blocking=True)
-        yd.copy_(yh, non_blocking=True)
-        res = ep.ep_layout(idd, E, R, w.align, w.capacity)
-        ep.ep_dispatch(res.handle, xd, w.fp8, recv, scales)
-        ep.ep_combine(res.handle, yd, twd, out)
-        oh.copy_(out, non_blocking=True)
-        return res.handle
+    def run(n_steps):
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_ready, comp_done, out_done = [], [], []
+        handles = []
+        for s in range(n_steps):
+            b = sets[s % 2]
+            with torch.cuda.stream(cin):
+                if s >= 2:
+                    cin.wait_event(comp_done[s - 2])      # set b no longer read by step s-2
+                b["x"].copy_(xh, non_blocking=True)
+                b["idx"].copy_(ih, non_blocking=True)
+                b["tw"].copy_(th, non_blocking=True)
+                b["y"].copy_(yh, non_blocking=True)
+                e = ev(); e.record(cin); in_ready.append(e)
+            comp.wait_event(in_ready[s])
+            if s >= 2:
+                comp.wait_event(out_done[s - 2])          # out of set b read back
+            res = ep.ep_layout(b["idx"], E, R, w.align, w.capacity)
+            ep.ep_dispatch(res.handle, b["x"], w.fp8, b["recv"], b["scales"])
+            ep.ep_combine(res.handle, b["y"], b["tw"], b["out"])
+            handles.append(res.handle)
+            e = ev(); e.record(comp); comp_done.append(e)
+            with torch.cuda.stream(cout):
+                cout.wait_event(comp_done[s])
+                ohs[s % 2].copy_(b["out"], non_blocking=True)
+                e = ev(); e.record(cout); out_done.append(e)
+        comp.wait_event(out_done[-1])
+        return handles
 
     n_steps = max(3, min(args.steps, 10))
-    for _ in range(2):
-        step().free()
+    for h in run(2):
+        h.free()
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    handles = []
-    e0.record(stream)
-    for _ in range(n_steps):
-        handles.append(step())
-    e1.record(stream)
+    e0.record(comp)
+    cin.wait_event(e0)
+    handles = run(n_steps)
+    e1.record(comp)
     torch.cuda.synchronize()
     for h in handles:
         h.free()
     ms = reduce_max(e0.elapsed_time(e1) / n_steps, world)
     total = reduce_sum(nbytes["step"], world)
     return {"value": total / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
+            "pipelined": "2 deep: uploads, kernels and readback of neighbouring steps overlap"}
 
 
 def main():

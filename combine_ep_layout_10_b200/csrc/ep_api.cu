@@ -46,8 +46,6 @@ cudaError_t handle_pool(int device, cudaMemPool_t *out) {
     return cudaSuccess;
 }
 
-constexpr int kMaxChunkChannels = EP_DISPATCH_MAX_CHUNK;
-
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -248,9 +246,8 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
     if (st != EP_OK) return st;
     if (dev != h->device) return EP_ERR_INVALID_ARG;
 
-    const int align_ch = out_fp8 ? 128 : 8;
-    const int nchunks = (H + kMaxChunkChannels - 1) / kMaxChunkChannels;
-    const int chunk = (int)round_up((size_t)((H + nchunks - 1) / nchunks), align_ch);
+    int chunk, nchunks;
+    dispatch_chunking(h->T, H, out_fp8 ? 128 : 8, info.num_sms, &chunk, &nchunks);
 
     DispatchArgs a{};
     a.x = static_cast<const uint8_t *>(x);
@@ -264,7 +261,7 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
     a.num_sms = num_sms;
     a.T = h->T; a.k = h->k; a.H = H;
     a.chunk = chunk;
-    a.nchunks = (H + chunk - 1) / chunk;
+    a.nchunks = nchunks;
     if ((int64_t)h->T * a.nchunks >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.nunits = h->T * a.nchunks;
     cudaError_t e = launch_dispatch(a, stream);
@@ -671,9 +668,8 @@ ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const voi
     if (st != EP_OK) return st;
     if (dev != plan->device || dev != peers->device) return EP_ERR_INVALID_ARG;
 
-    const int align_ch = out_fp8 ? 128 : 8;
-    const int nchunks = (H + kMaxChunkChannels - 1) / kMaxChunkChannels;
-    const int chunk = (int)round_up((size_t)((H + nchunks - 1) / nchunks), align_ch);
+    int chunk, nchunks;
+    dispatch_chunking(plan->T, H, out_fp8 ? 128 : 8, info.num_sms, &chunk, &nchunks);
     DispatchArgs a{};
     a.x = static_cast<const uint8_t *>(x);
     a.x_scales = x_scales;
@@ -686,7 +682,7 @@ ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const voi
     a.num_sms = num_sms;
     a.T = plan->T; a.k = plan->k; a.H = H;
     a.chunk = chunk;
-    a.nchunks = (H + chunk - 1) / chunk;
+    a.nchunks = nchunks;
     if ((int64_t)plan->T * a.nchunks >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.nunits = plan->T * a.nchunks;
     return cuda_status(launch_dispatch_peer(a, stream));

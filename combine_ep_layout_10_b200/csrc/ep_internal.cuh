@@ -14,6 +14,12 @@
 #ifndef EP_DISPATCH_MAX_CHUNK     // dispatch: at most this many channels per work unit
 #define EP_DISPATCH_MAX_CHUNK 8192
 #endif
+#ifndef EP_DISPATCH_MIN_UNITS_PER_SM  // dispatch: split rows into more chunks until the grid has
+#define EP_DISPATCH_MIN_UNITS_PER_SM 0  // this many blocks per SM (small batches; 0 = off)
+#endif
+#ifndef EP_DISPATCH_MIN_CHUNK     // dispatch: ... but never below this many channels per block
+#define EP_DISPATCH_MIN_CHUNK 512
+#endif
 #ifndef EP_DISPATCH_STORE_CS      // dispatch: evict-first (.cs) stores of the receive rows
 #define EP_DISPATCH_STORE_CS 0
 #endif
@@ -285,6 +291,28 @@ struct PlanArgs {
     int32_t *pre, *offs, *recv_seg, *recv_cnt;
     uint32_t *err;
 };
+
+// Work units of a dispatch: each token's H channels split into nchunks
+// chunks of `chunk` channels (a multiple of align_ch: 128 for FP8 groups, 8
+// for BF16 vectors), at most EP_DISPATCH_MAX_CHUNK each.  A small batch is
+// split further, down to EP_DISPATCH_MIN_CHUNK channels, until T * nchunks
+// reaches EP_DISPATCH_MIN_UNITS_PER_SM blocks per SM.
+inline void dispatch_chunking(int T, int H, int align_ch, int num_sms, int *chunk, int *nchunks) {
+    int n = (H + EP_DISPATCH_MAX_CHUNK - 1) / EP_DISPATCH_MAX_CHUNK;
+    const long long want_units = (long long)EP_DISPATCH_MIN_UNITS_PER_SM * num_sms;
+    if (T > 0 && (long long)T * n < want_units) {
+        const int min_chunk = EP_DISPATCH_MIN_CHUNK > align_ch ? EP_DISPATCH_MIN_CHUNK : align_ch;
+        int max_n = H / min_chunk;
+        if (max_n < 1) max_n = 1;
+        long long want = (want_units + T - 1) / T;
+        if (want > max_n) want = max_n;
+        if (want > n) n = (int)want;
+    }
+    int c = (H + n - 1) / n;
+    c = (c + align_ch - 1) / align_ch * align_ch;
+    *chunk = c;
+    *nchunks = (H + c - 1) / c;
+}
 
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
