@@ -83,3 +83,41 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(ep, "LIB_PATH", "/nonexistent/libep_b200.so")
     with pytest.raises(RuntimeError, match="missing"):
         ep.lib()
+
+
+def test_peer_max_recv_rows(L):
+    # every slot of every rank may land on one rank, plus alignment slack per owned expert
+    assert ep.ep_peer_max_recv_rows(8 * 8192, 8, 256, 8) == 8 * 8192 * 8
+    assert ep.ep_peer_max_recv_rows(1000, 8, 256, 8, 4) == 8000 + 32 * 3
+    assert ep.ep_peer_max_recv_rows(1000, 8, 256, 8, 1, 128) == 32 * 128
+    assert ep.ep_peer_max_recv_rows(1000, 8, 255, 8) == 0      # E % world
+    assert ep.ep_peer_max_recv_rows(-1, 8, 256, 8) == 0
+
+
+def test_multi_gpu_argument_errors_on_host(L):
+    P = ctypes.c_void_p
+    out = P()
+    fake = P(256)   # never dereferenced: validation fails first
+    INV = ep.EP_ERR_INVALID_ARG
+    # plan: no handle / no output slot
+    assert L.ep_plan_create(None, fake, fake, 0, 2, 1, 0, 64, ctypes.byref(out), None) == INV
+    assert L.ep_plan_create(fake, fake, fake, 0, 2, 1, 0, 64, None, None) == INV
+    # peers: empty group, missing or misaligned receive buffers
+    assert L.ep_peers_create(0, None, None, None, None, 64, ctypes.byref(out)) == INV
+    assert L.ep_peers_create(2, None, None, None, None, 64, ctypes.byref(out)) == INV
+    two = (P * 2)(256, 256 + 8)                                # second one not 16-byte aligned
+    assert L.ep_peers_create(2, two, None, None, None, 64, ctypes.byref(out)) == INV
+    nul = (P * 2)(256, None)
+    assert L.ep_peers_create(2, nul, None, None, None, 64, ctypes.byref(out)) == INV
+    # peer calls with no plan or table
+    assert L.ep_dispatch_peer(None, None, fake, None, 128, 0, 1, 0, None) == INV
+    assert L.ep_combine_peer(None, None, None, 128, fake, 0, None) == INV
+    assert L.ep_combine_backward_peer(None, None, fake, fake, 128, None, None) == INV
+    # IPC: null arguments
+    h = ctypes.create_string_buffer(ep.EP_IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64()
+    assert L.ep_ipc_export(None, h, ctypes.byref(off)) == INV
+    assert L.ep_ipc_import(None, 0, ctypes.byref(out)) == INV
+    assert L.ep_ipc_release(None, 0) == INV
+    assert L.ep_plan_check(None, None) == INV
+    assert L.ep_dispatch_topk(None, None, None, None, None, 0, None) == INV
