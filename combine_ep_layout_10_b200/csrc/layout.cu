@@ -37,10 +37,67 @@ __device__ __forceinline__ void load_words(int32_t *dst, const int32_t *src, int
         const int n4 = n >> 2;
         const int4 *s4 = reinterpret_cast<const int4 *>(src);
         int4 *d4 = reinterpret_cast<int4 *>(dst);
-        for (int i = threadIdx.x; i < n4; i += blockDim.x) d4[i] = __ldg(s4 + i);
+        // Batches of kBatch 16-byte loads per thread are all issued before any
+        // is stored, so a CTA's copy takes a few L2 round trips, not one per vector.
+        constexpr int kBatch = 8;
+        const int stride = blockDim.x;
+        for (int i0 = threadIdx.x; i0 < n4; i0 += kBatch * stride) {
+            int4 v[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int i = i0 + b * stride;
+                if (i < n4) v[b] = __ldg(s4 + i);
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int i = i0 + b * stride;
+                if (i < n4) d4[i] = v[b];
+            }
+        }
         for (int i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) dst[i] = __ldg(src + i);
     } else {
         for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = __ldg(src + i);
+    }
+}
+
+// is_token_in_rank rows of ntok consecutive tokens (one contiguous block of
+// ntok * R bytes at dst) from their rank bitmasks in shared memory (RW =
+// ceil(R / 32) words per token), by the whole CTA.  16-byte stores of 16
+// flags when dst and R allow (16 rank bits never straddle a mask word), else
+// 4-byte stores of 4 flags, else bytes.
+__device__ __forceinline__ void write_in_rank_rows(uint8_t *dst, const uint32_t *mask_s, int ntok, int R) {
+    const int RW = (R + 31) >> 5;
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(dst);
+    if ((addr & 15u) == 0 && (R & 15) == 0) {
+        const int per_row = R >> 4;
+        uint4 *d16 = reinterpret_cast<uint4 *>(dst);
+        for (int v = threadIdx.x; v < ntok * per_row; v += blockDim.x) {
+            const int tl = v / per_row;
+            const int f0 = (v - tl * per_row) * 16;
+            const uint32_t m = mask_s[tl * RW + (f0 >> 5)] >> (f0 & 31);
+            uint32_t q[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t b = m >> (4 * j);
+                q[j] = (b & 1u) | ((b & 2u) << 7) | ((b & 4u) << 14) | ((b & 8u) << 21);
+            }
+            d16[v] = make_uint4(q[0], q[1], q[2], q[3]);
+        }
+    } else if ((addr & 3u) == 0 && (R & 3) == 0) {
+        const int per_row = R >> 2;
+        uint32_t *d4 = reinterpret_cast<uint32_t *>(dst);
+        for (int v = threadIdx.x; v < ntok * per_row; v += blockDim.x) {
+            const int tl = v / per_row;
+            const int f0 = (v - tl * per_row) * 4;
+            const uint32_t b = mask_s[tl * RW + (f0 >> 5)] >> (f0 & 31);
+            d4[v] = (b & 1u) | ((b & 2u) << 7) | ((b & 4u) << 14) | ((b & 8u) << 21);
+        }
+    } else {
+        for (int i = threadIdx.x; i < ntok * R; i += blockDim.x) {
+            const int tl = i / R;
+            const int r = i - tl * R;
+            dst[i] = (uint8_t)((mask_s[tl * RW + (r >> 5)] >> (r & 31)) & 1u);
+        }
     }
 }
 
@@ -95,30 +152,8 @@ __global__ void __launch_bounds__(kCountThreads) layout_count_kernel(LayoutArgs 
         }
         __syncthreads();
 
-        if (a.out_in_rank != nullptr) {
-            const int nflags = ns * a.R;
-            uint8_t *dst = a.out_in_rank + (int64_t)(t0 + sb) * a.R;
-            if ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0 && (a.R & 3) == 0) {
-                // One warp per token row; lane w writes flags 4w..4w+3 as one word
-                // (a multiple of 4 never straddles a 32-bit mask word).
-                const int words = a.R >> 2;
-                const int lane = threadIdx.x & 31;
-                for (int tl = threadIdx.x >> 5; tl < ns; tl += blockDim.x >> 5) {
-                    uint32_t *dw = reinterpret_cast<uint32_t *>(dst + (int64_t)tl * a.R);
-                    const uint32_t *mrow = mask_s + tl * RW;
-                    for (int w4 = lane; w4 < words; w4 += 32) {
-                        const uint32_t m = mrow[w4 >> 3] >> ((w4 & 7) * 4);
-                        dw[w4] = (m & 1u) | ((m & 2u) << 7) | ((m & 4u) << 14) | ((m & 8u) << 21);
-                    }
-                }
-            } else {
-                for (int i = threadIdx.x; i < nflags; i += blockDim.x) {
-                    const int tl = i / a.R;
-                    const int r = i - tl * a.R;
-                    dst[i] = (uint8_t)((mask_s[tl * RW + (r >> 5)] >> (r & 31)) & 1u);
-                }
-            }
-        }
+        if (a.out_in_rank != nullptr)
+            write_in_rank_rows(a.out_in_rank + (int64_t)(t0 + sb) * a.R, mask_s, ns, a.R);
         __syncthreads();
     }
 
@@ -437,13 +472,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutArgs 
     if (a.out_rank_tok != nullptr)
         for (int r = threadIdx.x; r < R; r += blockDim.x) a.out_rank_tok[r] = rcnt_s[r];
     if (threadIdx.x == 0) *a.err = (bad ? kErrBadExpertId : 0u) | (over ? kErrCapacity : 0u);
-    if (a.out_in_rank != nullptr) {
-        for (int i = threadIdx.x; i < a.T * R; i += blockDim.x) {
-            const int t = i / R;
-            const int r = i - t * R;
-            a.out_in_rank[i] = (uint8_t)((mask_s[t * RW + (r >> 5)] >> (r & 31)) & 1u);
-        }
-    }
+    if (a.out_in_rank != nullptr) write_in_rank_rows(a.out_in_rank, mask_s, a.T, R);
     if (gridDim.x == 1) {
         // Packed mode: every row starts as padding (-1); the barrier orders
         // the fill before the valid rows are written over it below.

@@ -88,6 +88,7 @@ LAYOUT_EDGE = [
     (5000, 2, 16, 4, 1, 1024, 0),     # padded, tiled path (more than 8192 slots)
     (8193, 1, 8, 2, 1, 0, -1),        # one slot past the one-CTA limit
     (8192, 1, 8, 2, 1, 0, -1),        # exactly at the one-CTA limit
+    (9000, 2, 96, 48, 1, 0, -1),      # tiled, 16-flag vectors across mask-word halves
 ]
 
 
