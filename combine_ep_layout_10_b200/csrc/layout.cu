@@ -189,6 +189,11 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     if (a.ids_in_smem) load_words(ids_s, a.topk_idx + s0, nslots);
     load_words(mat, a.tile_cnt, NT * E);
     if (tile == 0) load_words(rmat, a.tile_rank, NT * R);
+    // CTA 0 also reads every tile's bad-id flag here, so the round trip
+    // overlaps the matrix load instead of delaying its publish step.
+    uint32_t tile_bad = 0u;
+    if (tile == 0)
+        for (int t = threadIdx.x; t < NT; t += blockDim.x) tile_bad |= __ldg(a.tile_err + t);
     for (int i = threadIdx.x; i < W * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
 
@@ -242,9 +247,7 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
                 a.out_rank_tok[r] = s;
             }
         }
-        uint32_t bad = 0u;
-        for (int t = threadIdx.x; t < NT; t += blockDim.x) bad |= __ldg(a.tile_err + t);
-        bad = __syncthreads_or(bad != 0u) ? kErrBadExpertId : 0u;
+        const uint32_t bad = __syncthreads_or(tile_bad != 0u) ? kErrBadExpertId : 0u;
         // The layout (re)initialises the handle's error word.
         if (threadIdx.x == 0) *a.err = bad | (over ? kErrCapacity : 0u);
     }
