@@ -1,6 +1,7 @@
 // ep_api.cu -- the C ABI declared in include/ep.h: argument validation,
-// handle ownership and kernel launches.  Every step of the data path runs in
-// the kernels of layout.cu, dispatch.cu and combine.cu; nothing here touches
+// ownership of handles, plans and peer tables, CUDA IPC, and kernel launches.
+// Every step of the data path runs in the kernels of layout.cu, dispatch.cu,
+// combine.cu, backward.cu, recv_topk.cu and plan.cu; nothing here touches
 // tensor data on the host.
 #include <algorithm>
 #include <cstdlib>

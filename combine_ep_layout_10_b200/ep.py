@@ -1,12 +1,17 @@
 """Python binding of the C ABI in include/ep.h (libep_b200.so).
 
-Argument marshalling only: every step of layout, dispatch and combine runs in
-the library's CUDA kernels.  PyTorch supplies device memory and the current
-stream.  There is no fallback: if the CUDA library is missing or the device is
-not an sm_100 part, the calls raise.
+Argument marshalling only: every step of layout, dispatch, combine, their
+backward pair and the multi-GPU plan runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream.  There is no
+fallback: if the CUDA library is missing or the device is not an sm_100 part,
+the calls raise.
 
 The names follow the C ABI: ep_max_recv_rows, ep_layout, ep_dispatch,
-ep_combine, ep_handle_free (plus the handle accessors).
+ep_combine, ep_handle_free (plus the handle accessors), the option, backward
+and per-row calls (ep_dispatch_ex, ep_combine_ex, ep_dispatch_backward,
+ep_combine_backward, ep_dispatch_topk, ep_layout_noalloc) and the multi-GPU
+calls (ep_plan_create, Peers, ep_dispatch_peer, ep_combine_peer,
+ep_combine_backward_peer, ipc_export / ipc_import / ipc_release).
 """
 from __future__ import annotations
 
