@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-cpu-baseline] [--no-e2e] [--no-decode]
-                    [--no-backward] [--no-overlap] [--no-ranks]
+                    [--no-backward] [--no-overlap] [--no-ranks] [--ep]
 
 A step is one pass of the whole path over one batch: ep_layout (2 kernels),
 ep_dispatch (FP8 e4m3 or BF16), ep_combine (BF16), all through the C ABI.
@@ -17,6 +17,10 @@ steps; K timed steps bracketed by barrier + synchronize; max over ranks.
 value = algorithmic bytes of all ranks' steps / time (GB/s).  Multi-GPU runs
 are independent replicas (each rank its own batch, seed + rank): the path
 has no exchange step on one node's virtual ranks, so there is no collective.
+
+`--ep` adds expert parallelism across the job's GPUs (peer dispatch and
+combine between the ranks, NCCL collectives between the phases) as an extra
+object of the same line.
 
 `--impl reference` times the CPU oracle (the plain single-threaded C
 implementation under oracle/) on a bounded sample of the same workload.
@@ -69,6 +73,8 @@ def parse():
     p.add_argument("--no-backward", action="store_true")
     p.add_argument("--no-overlap", action="store_true")
     p.add_argument("--no-ranks", action="store_true")
+    p.add_argument("--ep", action="store_true",
+                   help="also run expert parallelism across the job's GPUs (peer stores/loads)")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
 
@@ -193,6 +199,24 @@ class ClockSampler:
 # distributed plumbing (replicas only)
 # ---------------------------------------------------------------------------
 
+class _StdoutToStderr:
+    """Sends file descriptor 1 to stderr for a while: NCCL prints its version
+    line on stdout when a communicator is created, and stdout must carry
+    only the JSON result line."""
+
+    def __enter__(self):
+        sys.stdout.flush()
+        self.saved = os.dup(1)
+        os.dup2(2, 1)
+        return self
+
+    def __exit__(self, *exc):
+        sys.stdout.flush()
+        os.dup2(self.saved, 1)
+        os.close(self.saved)
+        return False
+
+
 def dist_setup(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -202,8 +226,9 @@ def dist_setup(n_gpus: int):
     if world > 1:
         import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        with _StdoutToStderr():
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     return world, rank, local
@@ -525,6 +550,10 @@ def run_ours(args, w):
     if world == 1 and not args.no_ranks:
         ranks = run_ranks_emulated(w, dev, ep, flush_l2)
 
+    ep_gpus = None
+    if args.ep:
+        ep_gpus = run_ep_across_gpus(args, w, world, rank, local)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed)
@@ -538,6 +567,7 @@ def run_ours(args, w):
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "decode": decode, "backward": backward, "overlap": overlap, "ranks_emulated": ranks,
+            "ep_across_gpus": ep_gpus,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "wall_s": wall,
             "host_us_per_step": host_s * 1e6,
         }
@@ -749,6 +779,83 @@ def run_ranks_emulated(w, dev, ep, flush_l2, worlds=(1, 8), steps: int = 10) -> 
         del recv, sc, ys
         torch.cuda.empty_cache()
     return out
+
+
+NVLINK_PEER_GBS = 770.0   # measured peer copy bandwidth per direction per GPU on this machine's B200s
+
+
+def run_ep_across_gpus(args, w, world, rank, local, steps: int = 10) -> dict:
+    """Expert parallelism across the job's GPUs (opt-in, --ep).  Every rank
+    holds its own batch of the workload's T tokens, the E experts are split
+    over the W ranks, and a step is the multi-GPU protocol of EpGroup: local
+    layout, count all-gather and plan; dispatch by peer stores into the
+    owners' receive buffers; combine by peer loads from the owners' expert
+    outputs; NCCL collectives between.  Device time per step is the max over
+    ranks.  NVLink bytes are the rows (plus FP8 scales) whose owner is another
+    rank, each way; with W = 1 every row is local."""
+    import socket
+    import torch.distributed as dist
+    from combine_ep_layout_10_b200 import ep, group
+    created = False
+    if not dist.is_initialized():
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        with _StdoutToStderr():
+            dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        created = True
+    dev = torch.device("cuda", local)
+    x_cpu, idx_cpu, tw_cpu = W.make_routing(w, replica_seed(args.seed, rank))
+    x, idx, tw = x_cpu.to(dev), idx_cpu.to(dev), tw_cpu.to(dev)
+    rows = ep.ep_peer_max_recv_rows(world * w.T, w.k, w.E, world)
+    g = group.EpGroup(w.E, w.H, rows, fp8=w.fp8)
+    gen = torch.Generator(device=dev).manual_seed(31 + rank)
+    g.y.copy_(torch.randn(rows, w.H, generator=gen, device=dev).to(torch.bfloat16))
+    for _ in range(max(args.warmup, 1)):
+        plan = g.dispatch(x, idx)
+        g.combine(plan, tw)
+        plan.free()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    plans = []
+    e0.record()
+    for _ in range(steps):
+        plan = g.dispatch(x, idx)
+        g.combine(plan, tw)
+        plans.append(plan)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(e0.elapsed_time(e1) / steps, world)
+    d = plans[0].export()["dst"]
+    owner = d[..., 0]
+    remote = int(((owner >= 0) & (owner != rank)).sum().item())     # rows this rank sends away
+    own = int((owner == rank).sum().item())                          # rows it keeps
+    recv = plans[0].recv_rows_host()
+    if any(p.check() != ep.EP_OK for p in plans):
+        raise SystemExit("ep_across_gpus: plan error")
+    for p in plans:
+        p.free()
+    g.close()
+    if created:
+        dist.destroy_process_group()
+    row_d = w.H * (1 if w.fp8 else 2) + (w.H // 128 * 4 if w.fp8 else 0)
+    row_c = w.H * 2
+    inbound = recv - own                                             # rows other ranks send here
+    # dispatch: out = rows sent, in = rows received; combine: the reverse, at bf16 width
+    d_link = reduce_max(float(max(remote, inbound) * row_d), world)
+    c_link = reduce_max(float(max(remote, inbound) * row_c), world)
+    floor_ms = (d_link + c_link) / (NVLINK_PEER_GBS * 1e9) * 1e3
+    return {"world": world, "tokens_per_rank": w.T, "ms_per_step": ms,
+            "rows_sent_this_rank": remote, "rows_received_from_peers_this_rank": inbound,
+            "nvlink_bytes_dispatch_busiest_rank": d_link, "nvlink_bytes_combine_busiest_rank": c_link,
+            "nvlink_floor_ms": floor_ms,
+            "frac_of_nvlink_floor": (floor_ms / ms) if ms > 0 and floor_ms > 0 else None,
+            "note": "per step: layout + all-gather + plan, peer dispatch, peer combine; floor = the "
+                    "busiest rank's larger direction per phase at the measured 770 GB/s peer bandwidth"}
 
 
 def run_overlap(w, dev, ep, idx_dev, x_dev, tw_dev, y_dev, flush_l2, reps: int = 10) -> dict:
