@@ -345,7 +345,7 @@ ep_status ep_layout_noalloc(const int32_t *topk_idx, int num_tokens, int num_top
  *
  * Peer memory: every rank's receive / scale / expert-output buffers must be
  * addressable from this process (ep_ipc_export / ep_ipc_import, or any other
- * mapping); only plain loads and stores reach them (no multicast). */
+ * mapping); only plain 16-byte loads and stores reach them. */
 
 /* Rows a rank may receive: total_tokens (all ranks) * k, plus
  * (E/W) * (expert_alignment - 1) of alignment slack; (E/W) * capacity when
