@@ -45,6 +45,9 @@
 #ifndef EP_BWD_MIN_BLOCKS         // combine backward: resident blocks per SM to plan registers for
 #define EP_BWD_MIN_BLOCKS 4
 #endif
+#ifndef EP_LAYOUT_LOAD_BATCH      // layout: 16-byte loads per thread in flight when staging counts
+#define EP_LAYOUT_LOAD_BATCH 8
+#endif
 #ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
 #define EP_USE_PDL 1
 #endif

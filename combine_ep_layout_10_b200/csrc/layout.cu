@@ -39,7 +39,7 @@ __device__ __forceinline__ void load_words(int32_t *dst, const int32_t *src, int
         int4 *d4 = reinterpret_cast<int4 *>(dst);
         // Batches of kBatch 16-byte loads per thread are all issued before any
         // is stored, so a CTA's copy takes a few L2 round trips, not one per vector.
-        constexpr int kBatch = 8;
+        constexpr int kBatch = EP_LAYOUT_LOAD_BATCH;
         const int stride = blockDim.x;
         for (int i0 = threadIdx.x; i0 < n4; i0 += kBatch * stride) {
             int4 v[kBatch];
