@@ -270,3 +270,39 @@ def test_peer_combine_backward(name, Ts, align, H):
                 yrow = ys[d[t, j, 0]][d[t, j, 1]].double().numpy()
                 lim = bound * np.abs(g64[t] * yrow).sum() + 1e-30
                 assert abs(float(gws[r][t, j]) - want_gw[r][t, j]) <= lim
+
+
+def test_metric_batch_over_eight_ranks_sampled():
+    """The benchmark's batch split over 8 emulated ranks of 1,024 tokens:
+    every slot's (owner, row) exactly the oracle's, every rank's segments and
+    counts too; FP8 rows and combined outputs exact on a sample of tokens
+    the oracle computes one by one."""
+    base = W.WORKLOADS["group_limited"]
+    Wr, Tr = 8, base.T // 8
+    parts = [W.make_routing(base.scaled(T=Tr), seed=7000 + r) for r in range(Wr)]
+    x_list = [p[0] for p in parts]
+    idx_list = [p[1] for p in parts]
+    w_list = [p[2] for p in parts]
+    em = Emulated(base.E, base.k, base.H, idx_list, True)
+    _, RL = MR.layout(idx_list, base.E, Wr)
+    check_plans(em, RL)
+    em.dispatch(x_list)
+    gy = torch.Generator(device=DEV).manual_seed(910)
+    for r in range(Wr):   # expert outputs drawn on the device; the checks read them back
+        em.y[r].copy_(torch.randn(em.recv_rows, base.H, generator=gy, device=DEV).to(torch.bfloat16))
+    outs = em.combine(w_list)
+    g = torch.Generator().manual_seed(12)
+    for s in range(Wr):
+        d = RL.destinations(s)
+        sample = torch.randperm(Tr, generator=g)[:8].tolist() + ([0, Tr - 1] if s in (0, Wr - 1) else [])
+        for t in sample:
+            q1, s1 = oracle.dispatch_fp8(x_list[s][t:t + 1], np.zeros((1, 1), np.int32), 1)
+            rows = []
+            for j in range(base.k):
+                o, row = int(d[t, j, 0]), int(d[t, j, 1])
+                assert (em.recv[o][row].cpu().numpy() == q1[0]).all()
+                assert (em.scales[o][row].cpu().numpy().view(np.uint32) == s1[0].view(np.uint32)).all()
+                rows.append(em.y[o][row].cpu())
+            want = oracle.combine(torch.stack(rows), w_list[s][t:t + 1].numpy(),
+                                  np.arange(base.k, dtype=np.int32)[None, :])
+            assert (u16(outs[s][t:t + 1]) == want).all()
