@@ -1,4 +1,4 @@
-"""The multi-GPU protocol end to end in two processes (GPU).
+"""The multi-GPU protocol end to end in separate processes (GPU).
 
 Two ranks of an EpGroup, each its own process with its own CUDA context,
 share their receive / scale / expert-output buffers through CUDA IPC and
@@ -29,13 +29,15 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, backend="gloo"):
     import sys
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    torch.cuda.set_device(0)
+    kw = {"device_id": torch.device("cuda", 0)} if backend == "nccl" else {}
+    dist.init_process_group(backend, rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60), **kw)
     result = {"rank": rank, "error": None}
     try:
         torch.cuda.set_device(0)
@@ -45,11 +47,12 @@ def _worker(rank, world, port, q):
         from combine_ep_layout_10_b200 import workloads as W
         base = W.WORKLOADS["prefill"]
         E, H, k = base.E, base.H, base.k
-        routed = [W.make_routing(base.scaled(T=T), seed=50 + r) for r, T in enumerate(TOKENS)]
+        tokens = TOKENS[:world]
+        routed = [W.make_routing(base.scaled(T=T), seed=50 + r) for r, T in enumerate(tokens)]
         x_list = [r[0] for r in routed]
         idx_list = [r[1] for r in routed]
         w_list = [r[2] for r in routed]
-        recv_rows = ep.ep_peer_max_recv_rows(sum(TOKENS), k, E, world)
+        recv_rows = ep.ep_peer_max_recv_rows(sum(tokens), k, E, world)
         g = group.EpGroup(E, H, recv_rows, fp8=True)
         _, RL = MR.layout(idx_list, E, world)
         n = RL.recv_rows(rank)
@@ -73,12 +76,12 @@ def _worker(rank, world, port, q):
         want = MR.combine(RL, ys, w_list)[rank]
         result["combine"] = bool((out.view(torch.int16).cpu().numpy().view(np.uint16) == want).all())
         # second step: same routing (cached plan), new hidden states
-        x2 = [W.make_x(base.scaled(T=T), 1000 + r) for r, T in enumerate(TOKENS)]
+        x2 = [W.make_x(base.scaled(T=T), 1000 + r) for r, T in enumerate(tokens)]
         g.dispatch(x2[rank].cuda(), plan=plan)
         torch.cuda.synchronize()
         result["cached"] = check_recv(x2)
         # backward: combine's (gradient rows to the owners), then dispatch's
-        gos = [W.make_x(base.scaled(T=T), 2000 + r) for r, T in enumerate(TOKENS)]
+        gos = [W.make_x(base.scaled(T=T), 2000 + r) for r, T in enumerate(tokens)]
         gw = g.combine_backward(plan, gos[rank].cuda(), w_list[rank].cuda())
         torch.cuda.synchronize()
         want_gy, want_gw = MR.combine_backward(RL, gos, ys, w_list)
@@ -102,16 +105,15 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_processes_share_buffers_over_ipc():
+def _run(world, backend):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     from combine_ep_layout_10_b200 import build
     build.build()
-    world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, backend)) for r in range(world)]
     for p in procs:
         p.start()
     results = []
@@ -127,3 +129,14 @@ def test_two_processes_share_buffers_over_ipc():
         assert r["error"] is None, r
         assert r["dispatch"] and r["rows"] and r["combine"] and r["cached"], r
         assert r["combine_bwd"] and r["dispatch_bwd"], r
+
+
+def test_two_processes_share_buffers_over_ipc():
+    _run(2, "gloo")
+
+
+def test_single_rank_group_over_nccl():
+    """The NCCL branch of EpGroup (device-ordered all-reduce barriers and the
+    all_gather_into_tensor of the counts) with one rank, whose peer table is
+    its own buffers."""
+    _run(1, "nccl")
