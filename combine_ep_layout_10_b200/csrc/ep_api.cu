@@ -118,7 +118,7 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     ep_status st = current_device(&dev, &info);
     if (st != EP_OK) return st;
 
-    const LayoutGeometry geo = layout_geometry(T, k, E, R);
+    const LayoutGeometry geo = layout_geometry(T, k, E, R, C);
     const int ntiles = geo.ntiles;
 
     // One stream-ordered allocation, every array 256-byte aligned.

@@ -48,6 +48,17 @@
 #ifndef EP_LAYOUT_LOAD_BATCH      // layout: 16-byte loads per thread in flight when staging counts
 #define EP_LAYOUT_LOAD_BATCH 8
 #endif
+// Layout: the one-CTA path up to this many slots.  Measured on B200 (E = 256,
+// k = 8): one CTA takes 13.2 / 16.0 / 21.4 / 29.7 us at 1K / 2K / 4K / 8K
+// slots, the two tiled kernels 17.4 / 16.8 / 15.3 / 15.3 us, so packed
+// layouts switch at 2K slots.  Padded layouts stay on one CTA up to 8K: its
+// helper CTAs spread the padding fill (decode shape: 12.5 us, tiled 21.5 us).
+#ifndef EP_LAYOUT_SMALL_MAX_SLOTS
+#define EP_LAYOUT_SMALL_MAX_SLOTS 2048
+#endif
+#ifndef EP_LAYOUT_SMALL_MAX_SLOTS_PADDED
+#define EP_LAYOUT_SMALL_MAX_SLOTS_PADDED 8192
+#endif
 #ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
 #define EP_USE_PDL 1
 #endif
@@ -156,7 +167,7 @@ inline int layout_pos_smem_words(int ntiles, int E, int R, int pos_warps, int id
     return align4(ntiles * E) + align4(ntiles * R) + 2 * align4(E) + align4(E + 1) +
            align4(pos_warps * E) + id_words;
 }
-inline LayoutGeometry layout_geometry(int T, int k, int E, int R) {
+inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) {
     LayoutGeometry g;
     g.tile_tokens = 128;
     while ((int64_t)((T + g.tile_tokens - 1) / g.tile_tokens) * (E + R) > kLayoutMatWords &&
@@ -169,7 +180,8 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R) {
     const int64_t id_words = (int64_t)g.tile_tokens * k;
     g.ids_in_smem = id_words <= 8192 &&
                     layout_pos_smem_words(g.ntiles, E, R, g.pos_warps, (int)id_words) <= 50000;
-    g.small = T > 0 && (int64_t)T * k <= 8192 && E <= 512 &&
+    const int64_t small_max = capacity > 0 ? EP_LAYOUT_SMALL_MAX_SLOTS_PADDED : EP_LAYOUT_SMALL_MAX_SLOTS;
+    g.small = T > 0 && (int64_t)T * k <= small_max && E <= 512 &&
               layout_small_smem_words(T, k, E, R) <= 40000;
     return g;
 }

@@ -333,9 +333,11 @@ __device__ __forceinline__ void fill_minus_one(int32_t *dst, int64_t n) {
 // ---------------------------------------------------------------------------
 // Small problems: the whole layout in one CTA of 1024 threads
 // ---------------------------------------------------------------------------
-// With at most 8192 slots, one CTA holds every id, the expert histogram, the
-// per-warp counts and the rank bitmasks in shared memory, so counts, segments
-// and positions need no second kernel and no count matrices in global memory.
+// With at most 2048 slots (8192 in padded mode; the thresholds and their
+// measurements are in ep_internal.cuh), one CTA holds every id, the expert
+// histogram, the per-warp counts and the rank bitmasks in shared memory, so
+// counts, segments and positions need no second kernel and no count matrices
+// in global memory.
 // The 32 warps own contiguous slot ranges; ranks inside an expert come from
 // __match_any_sync + popc plus a prefix over the warps, as in the tiled path.
 constexpr int kSmallThreads = 1024;

@@ -83,7 +83,7 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
         return EP_ERR_INVALID_ARG;
 
     // Same tile geometry as ep_layout.
-    const LayoutGeometry geo = layout_geometry(T, k, E, R);
+    const LayoutGeometry geo = layout_geometry(T, k, E, R, C);
     const int ntiles = geo.ntiles;
 
     // Scratch words (16-byte aligned blocks): tile_cnt, tile_rank, per-expert
