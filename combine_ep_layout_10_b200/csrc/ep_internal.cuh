@@ -56,6 +56,9 @@
 #ifndef EP_LAYOUT_SMALL_MAX_SLOTS
 #define EP_LAYOUT_SMALL_MAX_SLOTS 2048
 #endif
+#ifndef EP_LAYOUT_TILE_TOKENS     // layout: tokens per tile of the tiled path (doubled for large T)
+#define EP_LAYOUT_TILE_TOKENS 128
+#endif
 #ifndef EP_LAYOUT_SMALL_MAX_SLOTS_PADDED
 #define EP_LAYOUT_SMALL_MAX_SLOTS_PADDED 8192
 #endif
@@ -169,7 +172,7 @@ inline int layout_pos_smem_words(int ntiles, int E, int R, int pos_warps, int id
 }
 inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) {
     LayoutGeometry g;
-    g.tile_tokens = 128;
+    g.tile_tokens = EP_LAYOUT_TILE_TOKENS;
     while ((int64_t)((T + g.tile_tokens - 1) / g.tile_tokens) * (E + R) > kLayoutMatWords &&
            g.tile_tokens < (1 << 29))
         g.tile_tokens *= 2;
