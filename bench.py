@@ -992,9 +992,26 @@ def run_e2e(args, w, dev, ep, x_cpu, idx_cpu, tw_cpu, y_dev, nbytes, world):
         h.free()
     ms = reduce_max(e0.elapsed_time(e1) / n_steps, world)
     total = reduce_sum(nbytes["step"], world)
+    # The link this number is bound by: one plain pinned upload of the same
+    # bytes (the largest input), timed alone on the copy stream.
+    big = sets[0]["y"]
+    up = []
+    for _ in range(3):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(cin)
+        big.copy_(yh, non_blocking=True)
+        b.record(cin)
+        torch.cuda.synchronize()
+        up.append(a.elapsed_time(b))
+    h2d_gbs = yh.numel() * yh.element_size() / (min(up) / 1e3) / 1e9
+    step_h2d_gbs = h2d / (ms / 1e3) / 1e9
     return {"value": total / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
-            "pipelined": "2 deep: uploads, kernels and readback of neighbouring steps overlap"}
+            "pipelined": "2 deep: uploads, kernels and readback of neighbouring steps overlap",
+            "roofline": {"bound": "pcie_h2d", "achieved": step_h2d_gbs, "peak": h2d_gbs, "unit": "GB/s",
+                         "frac": step_h2d_gbs / h2d_gbs,
+                         "peak_source": "one pinned %.0f MB upload timed alone" % (yh.numel() * yh.element_size() / 1e6)}}
 
 
 def main():
