@@ -49,12 +49,20 @@
 #define EP_LAYOUT_LOAD_BATCH 8
 #endif
 // Layout: the one-CTA path up to this many slots.  Measured on B200 (E = 256,
-// k = 8): one CTA takes 13.2 / 16.0 / 21.4 / 29.7 us at 1K / 2K / 4K / 8K
-// slots, the two tiled kernels 17.4 / 16.8 / 15.3 / 15.3 us, so packed
-// layouts switch at 2K slots.  Padded layouts stay on one CTA up to 8K: its
-// helper CTAs spread the padding fill (decode shape: 12.5 us, tiled 21.5 us).
+// k = 8): one CTA takes 12.3 / 16.2 / 21.4 / 29.7 us at 1K / 2K / 4K / 8K
+// slots, the two tiled kernels (with the position kernel sized to its tile)
+// about 15.3 us at every size from 2K slots up, so packed layouts switch at
+// 1.5K slots.  Padded layouts stay on one CTA up to 8K: its helper CTAs
+// spread the padding fill (decode shape: 12.5 us, tiled 21.5 us).
 #ifndef EP_LAYOUT_SMALL_MAX_SLOTS
-#define EP_LAYOUT_SMALL_MAX_SLOTS 2048
+#define EP_LAYOUT_SMALL_MAX_SLOTS 1536
+#endif
+// Layout: the position kernel runs about 2 tile slots per thread (rounded to
+// whole warps, 256..EP_LAYOUT_POS_MAX_THREADS).  Measured on B200: 256 / 512 /
+// 1024 threads gave 17.4 / 15.3 / 17.4 us at the metric shape (1024-slot
+// tiles) and 21.5 / 21.5 / 19.4 us at large-skewed (2048-slot tiles).
+#ifndef EP_LAYOUT_POS_MAX_THREADS
+#define EP_LAYOUT_POS_MAX_THREADS 1024
 #endif
 #ifndef EP_LAYOUT_TILE_TOKENS     // layout: tokens per tile of the tiled path (doubled for large T)
 #define EP_LAYOUT_TILE_TOKENS 128
@@ -157,7 +165,7 @@ __host__ __device__ constexpr int align4(int n) { return (n + 3) & ~3; }
 // shared memory when they fit.
 constexpr int kLayoutMatWords = 24576;
 struct LayoutGeometry {
-    int tile_tokens, ntiles, sub_tokens, pos_warps;
+    int tile_tokens, ntiles, sub_tokens, pos_warps, pos_threads;
     bool ids_in_smem;  // the position kernel stages the tile's ids in shared memory
     bool small;        // the whole layout fits one CTA (layout_small_kernel)
 };
@@ -179,7 +187,10 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) 
     g.ntiles = (T + g.tile_tokens - 1) / g.tile_tokens;
     const int rw = (R + 31) / 32;
     g.sub_tokens = 12288 / rw < g.tile_tokens ? 12288 / rw : g.tile_tokens;
-    g.pos_warps = 12288 / E >= 8 ? 8 : (12288 / E > 0 ? 12288 / E : 1);
+    int64_t pt = ((int64_t)g.tile_tokens * k / 2 + 31) / 32 * 32;
+    g.pos_threads = (int)(pt < 256 ? 256 : pt > EP_LAYOUT_POS_MAX_THREADS ? EP_LAYOUT_POS_MAX_THREADS : pt);
+    const int pos_warps = g.pos_threads / 32;
+    g.pos_warps = 12288 / E >= pos_warps ? pos_warps : (12288 / E > 0 ? 12288 / E : 1);
     const int64_t id_words = (int64_t)g.tile_tokens * k;
     g.ids_in_smem = id_words <= 8192 &&
                     layout_pos_smem_words(g.ntiles, E, R, g.pos_warps, (int)id_words) <= 50000;
@@ -192,7 +203,7 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) 
 struct LayoutArgs {
     const int32_t *topk_idx;
     int T, k, E, R, epr, align, capacity;
-    int tile_tokens, ntiles, sub_tokens, pos_warps;
+    int tile_tokens, ntiles, sub_tokens, pos_warps, pos_threads;
     bool ids_in_smem, small;
     int64_t n_rows;
     int32_t *pos, *src_idx, *seg, *rank_off, *cnt, *tile_cnt, *tile_rank;

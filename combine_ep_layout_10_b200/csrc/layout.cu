@@ -29,7 +29,7 @@ namespace ep {
 namespace {
 
 constexpr int kCountThreads = 256;
-constexpr int kPosThreads = 256;
+constexpr int kPosThreads = EP_LAYOUT_POS_MAX_THREADS;  // launch bound; the launch uses a.pos_threads
 
 // Copy n int32 words global -> shared (16-byte vectors when both are aligned).
 __device__ __forceinline__ void load_words(int32_t *dst, const int32_t *src, int n) {
@@ -333,7 +333,7 @@ __device__ __forceinline__ void fill_minus_one(int32_t *dst, int64_t n) {
 // ---------------------------------------------------------------------------
 // Small problems: the whole layout in one CTA of 1024 threads
 // ---------------------------------------------------------------------------
-// With at most 2048 slots (8192 in padded mode; the thresholds and their
+// With at most 1536 slots (8192 in padded mode; the thresholds and their
 // measurements are in ep_internal.cuh), one CTA holds every id, the expert
 // histogram, the per-warp counts and the rank bitmasks in shared memory, so
 // counts, segments and positions need no second kernel and no count matrices
@@ -580,7 +580,7 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s) {
     if ((err = ensure_dyn_smem(layout_pos_kernel, pos_smem, g_smem_pos)) != cudaSuccess) return err;
     if ((err = launch_kernel(layout_count_kernel, a.ntiles, kCountThreads, count_smem, s, a)) != cudaSuccess)
         return err;
-    return launch_kernel(layout_pos_kernel, a.ntiles, kPosThreads, pos_smem, s, a);
+    return launch_kernel(layout_pos_kernel, a.ntiles, a.pos_threads, pos_smem, s, a);
 }
 
 }  // namespace ep

@@ -86,8 +86,10 @@ LAYOUT_EDGE = [
     (64, 32, 4096, 4096, 1, 0, -1),   # maximum k, E, R
     (2048, 6, 96, 12, 8, 0, -1),      # E not a power of two
     (5000, 2, 16, 4, 1, 1024, 0),     # padded, tiled path (more than 8192 slots)
-    (2049, 1, 8, 2, 1, 0, -1),        # one slot past the packed one-CTA limit
-    (2048, 1, 8, 2, 1, 0, -1),        # exactly at the packed one-CTA limit
+    (1537, 1, 8, 2, 1, 0, -1),        # one slot past the packed one-CTA limit
+    (1536, 1, 8, 2, 1, 0, -1),        # exactly at the packed one-CTA limit
+    (2048, 8, 256, 64, 1, 0, -1),     # 16K slots: 16 tiles, position kernel at 512 threads
+    (1000, 8, 2048, 2048, 1, 0, -1),  # tiles doubled to 2K slots: position kernel at 1024 threads
     (1024, 8, 256, 64, 1, 0, -1),     # 8K slots packed: tiled
     (8193, 1, 8, 2, 1, 2048, 0),      # one slot past the padded one-CTA limit
     (8192, 1, 8, 2, 1, 2048, 0),      # exactly at the padded one-CTA limit
