@@ -104,7 +104,11 @@ template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
     __shared__ uint8_t *row_s[kMaxTopk];
     __shared__ float *srow_s[kMaxTopk];
+#if EP_DISPATCH_EARLY_TRIGGER
     pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
     const int tid = threadIdx.x;
     const bool leader = (tid & 7) == 0;
     // One unit per block unless the grid is capped (LOOP): then a grid stride.
@@ -167,7 +171,11 @@ template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) {
     __shared__ uint8_t *row_s[kMaxTopk];
     __shared__ float *srow_s[kMaxTopk];
+#if EP_DISPATCH_EARLY_TRIGGER
     pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
     const int tid = threadIdx.x;
     const bool leader = (tid & 7) == 0;
     const int G_row = a.H / 128;
@@ -204,7 +212,11 @@ template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchArgs a) {
     __shared__ uint8_t *row_s[kMaxTopk];
     __shared__ float *srow_s[kMaxTopk];
+#if EP_DISPATCH_EARLY_TRIGGER
     pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
     const int tid = threadIdx.x;
     // One unit per block unless the grid is capped (LOOP): then a grid stride.
     for (int u = blockIdx.x; u < a.nunits; u += gridDim.x) {

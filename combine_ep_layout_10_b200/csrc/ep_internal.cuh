@@ -57,18 +57,26 @@
 #ifndef EP_LAYOUT_SMALL_MAX_SLOTS
 #define EP_LAYOUT_SMALL_MAX_SLOTS 1536
 #endif
-// Layout: the position kernel runs about 2 tile slots per thread (rounded to
-// whole warps, 256..EP_LAYOUT_POS_MAX_THREADS).  Measured on B200: 256 / 512 /
-// 1024 threads gave 17.4 / 15.3 / 17.4 us at the metric shape (1024-slot
-// tiles) and 21.5 / 21.5 / 19.4 us at large-skewed (2048-slot tiles).
-#ifndef EP_LAYOUT_POS_MAX_THREADS
-#define EP_LAYOUT_POS_MAX_THREADS 1024
+// Layout: the tiled kernels run about 2 tile slots per thread (rounded to
+// whole warps, 256..EP_LAYOUT_TILE_MAX_THREADS).  Measured on B200 for the
+// position kernel: 256 / 512 / 1024 threads gave 17.4 / 15.3 / 17.4 us at the
+// metric shape (1024-slot tiles) and 21.5 / 21.5 / 19.4 us at large-skewed
+// (2048-slot tiles); the count kernel at 1024 threads took large-skewed from
+// 19.5 to 19.0 us and left the others unchanged.
+#ifndef EP_LAYOUT_TILE_MAX_THREADS
+#define EP_LAYOUT_TILE_MAX_THREADS 1024
 #endif
 #ifndef EP_LAYOUT_TILE_TOKENS     // layout: tokens per tile of the tiled path (doubled for large T)
 #define EP_LAYOUT_TILE_TOKENS 128
 #endif
 #ifndef EP_LAYOUT_SMALL_MAX_SLOTS_PADDED
 #define EP_LAYOUT_SMALL_MAX_SLOTS_PADDED 8192
+#endif
+#ifndef EP_LAYOUT_POS_EARLY_TRIGGER  // layout position kernel lets its dependents launch at its start
+#define EP_LAYOUT_POS_EARLY_TRIGGER 0
+#endif
+#ifndef EP_DISPATCH_EARLY_TRIGGER    // dispatch kernels let their dependents launch at their start
+#define EP_DISPATCH_EARLY_TRIGGER 1
 #endif
 #ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
 #define EP_USE_PDL 1
@@ -83,6 +91,15 @@ namespace ep {
 // completed and its memory is visible, so no input is read early.  It then
 // lets its own dependents be scheduled.  The saving is the launch latency
 // between back-to-back kernels.
+// Wait only: the kernel's dependents launch when it exits (for kernels whose
+// dependents can do nothing before it completes and whose early-launched
+// blocks would only take resources from it).
+__device__ __forceinline__ void pdl_wait() {
+#if EP_USE_PDL
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
 __device__ __forceinline__ void pdl_wait_then_trigger() {
 #if EP_USE_PDL
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -165,7 +182,7 @@ __host__ __device__ constexpr int align4(int n) { return (n + 3) & ~3; }
 // shared memory when they fit.
 constexpr int kLayoutMatWords = 24576;
 struct LayoutGeometry {
-    int tile_tokens, ntiles, sub_tokens, pos_warps, pos_threads;
+    int tile_tokens, ntiles, sub_tokens, pos_warps, tile_threads;
     bool ids_in_smem;  // the position kernel stages the tile's ids in shared memory
     bool small;        // the whole layout fits one CTA (layout_small_kernel)
 };
@@ -188,8 +205,8 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) 
     const int rw = (R + 31) / 32;
     g.sub_tokens = 12288 / rw < g.tile_tokens ? 12288 / rw : g.tile_tokens;
     int64_t pt = ((int64_t)g.tile_tokens * k / 2 + 31) / 32 * 32;
-    g.pos_threads = (int)(pt < 256 ? 256 : pt > EP_LAYOUT_POS_MAX_THREADS ? EP_LAYOUT_POS_MAX_THREADS : pt);
-    const int pos_warps = g.pos_threads / 32;
+    g.tile_threads = (int)(pt < 256 ? 256 : pt > EP_LAYOUT_TILE_MAX_THREADS ? EP_LAYOUT_TILE_MAX_THREADS : pt);
+    const int pos_warps = g.tile_threads / 32;
     g.pos_warps = 12288 / E >= pos_warps ? pos_warps : (12288 / E > 0 ? 12288 / E : 1);
     const int64_t id_words = (int64_t)g.tile_tokens * k;
     g.ids_in_smem = id_words <= 8192 &&
@@ -203,7 +220,7 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) 
 struct LayoutArgs {
     const int32_t *topk_idx;
     int T, k, E, R, epr, align, capacity;
-    int tile_tokens, ntiles, sub_tokens, pos_warps, pos_threads;
+    int tile_tokens, ntiles, sub_tokens, pos_warps, tile_threads;
     bool ids_in_smem, small;
     int64_t n_rows;
     int32_t *pos, *src_idx, *seg, *rank_off, *cnt, *tile_cnt, *tile_rank;

@@ -28,8 +28,8 @@
 namespace ep {
 namespace {
 
-constexpr int kCountThreads = 256;
-constexpr int kPosThreads = EP_LAYOUT_POS_MAX_THREADS;  // launch bound; the launch uses a.pos_threads
+constexpr int kCountThreads = EP_LAYOUT_TILE_MAX_THREADS;  // launch bound; the launch uses a.tile_threads
+constexpr int kPosThreads = EP_LAYOUT_TILE_MAX_THREADS;    // launch bound; the launch uses a.tile_threads
 
 // Copy n int32 words global -> shared (16-byte vectors when both are aligned).
 __device__ __forceinline__ void load_words(int32_t *dst, const int32_t *src, int n) {
@@ -180,7 +180,11 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     int32_t *ids_s = wcnt + align4(W * E);               // [tile_tokens * k] when a.ids_in_smem
     __shared__ int32_t warp_s[33];
 
+#if EP_LAYOUT_POS_EARLY_TRIGGER
     pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
     const int tile = blockIdx.x;
     const int t0 = tile * a.tile_tokens;
     const int nt = min(a.tile_tokens, a.T - t0);
@@ -578,9 +582,9 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s) {
     const size_t pos_smem = layout_pos_smem(a);
     if ((err = ensure_dyn_smem(layout_count_kernel, count_smem, g_smem_count)) != cudaSuccess) return err;
     if ((err = ensure_dyn_smem(layout_pos_kernel, pos_smem, g_smem_pos)) != cudaSuccess) return err;
-    if ((err = launch_kernel(layout_count_kernel, a.ntiles, kCountThreads, count_smem, s, a)) != cudaSuccess)
+    if ((err = launch_kernel(layout_count_kernel, a.ntiles, a.tile_threads, count_smem, s, a)) != cudaSuccess)
         return err;
-    return launch_kernel(layout_pos_kernel, a.ntiles, a.pos_threads, pos_smem, s, a);
+    return launch_kernel(layout_pos_kernel, a.ntiles, a.tile_threads, pos_smem, s, a);
 }
 
 }  // namespace ep

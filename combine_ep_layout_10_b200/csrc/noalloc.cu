@@ -112,7 +112,7 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
     a.ntiles = ntiles;
     a.sub_tokens = geo.sub_tokens;
     a.pos_warps = geo.pos_warps;
-    a.pos_threads = geo.pos_threads;
+    a.tile_threads = geo.tile_threads;
     a.ids_in_smem = geo.ids_in_smem;
     a.small = geo.small;
     a.n_rows = (int64_t)n_rows;
