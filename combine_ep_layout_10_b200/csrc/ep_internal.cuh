@@ -75,6 +75,9 @@
 #ifndef EP_LAYOUT_POS_EARLY_TRIGGER  // layout position kernel lets its dependents launch at its start
 #define EP_LAYOUT_POS_EARLY_TRIGGER 0
 #endif
+#ifndef EP_LAYOUT_COUNT_EARLY_TRIGGER  // layout count kernel lets the position kernel launch at its start
+#define EP_LAYOUT_COUNT_EARLY_TRIGGER 1
+#endif
 #ifndef EP_DISPATCH_EARLY_TRIGGER    // dispatch kernels let their dependents launch at their start
 #define EP_DISPATCH_EARLY_TRIGGER 1
 #endif

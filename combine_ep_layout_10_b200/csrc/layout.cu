@@ -114,7 +114,11 @@ __device__ __forceinline__ int tile_id(const LayoutArgs &a, const int32_t *ids_s
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kCountThreads) layout_count_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
+#if EP_LAYOUT_COUNT_EARLY_TRIGGER
     pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
     const int RW = (a.R + 31) >> 5;                                 // mask words per token
     int32_t *cnt_s = reinterpret_cast<int32_t *>(smem);             // [E]
     int32_t *rcnt_s = cnt_s + a.E;                                  // [R]
