@@ -21,6 +21,12 @@
 //      and a prefix over its warps, and writes pos[t][j] and src_idx[row].
 //      CTA 0 publishes counts, segments, rank slices, rank counts and the
 //      error word; the -1 fill of padding rows is spread over all CTAs.
+// Both run about two tile slots per thread (256..1024 threads; the rule and
+// its measurements are in ep_internal.cuh).  The position kernel lets
+// dispatch launch only when it exits: early-launched dispatch blocks would
+// only wait beside it and take its registers and warp slots.
+// Small problems take a third kernel instead, layout_small_kernel: the whole
+// layout in one CTA (plus padding-fill helpers in padded mode).
 #include <atomic>
 
 #include "ep_internal.cuh"
