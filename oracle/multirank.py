@@ -117,3 +117,25 @@ def combine_backward(RL: RankedLayout, grad_out_list, y_list, w_list):
     gy, gw = oracle.combine_backward(g, _concat_y(RL, y_list), w, RL.L.pos)
     return ([gy[RL.L.rank_off[r]:RL.L.rank_off[r + 1]] for r in range(RL.W)],
             [gw[b:b + T] for b, T in zip(RL.token_base, RL.T)])
+
+
+def dispatch_topk(RL: RankedLayout, idx_list, w_list):
+    """Per-row routing outputs on every owner rank: (recv_topk_idx int32,
+    recv_topk_weights float32, recv_src_rank int32, recv_slot int32), each
+    [recv_rows(r)]; recv_slot is the slot's flat index t*k + j on its source
+    rank.  Rows no slot fills get -1, 0, -1, -1."""
+    idx = np.concatenate([np.asarray(a, np.int32) for a in idx_list])
+    w = np.concatenate([np.asarray(a, np.float32) for a in w_list])
+    ri, rw, rs = oracle.dispatch_topk(idx, w, RL.L.pos, RL.L.n_rows)
+    k = RL.L.k
+    rank_of_token = np.repeat(np.arange(RL.W, dtype=np.int64), RL.T)   # concatenated token -> source rank
+    base = np.asarray(RL.token_base, np.int64)
+    out = []
+    for r in range(RL.W):
+        a, b = RL.L.rank_off[r], RL.L.rank_off[r + 1]
+        slot_g = rs[a:b].astype(np.int64)
+        filled = slot_g >= 0
+        src = np.where(filled, rank_of_token[np.where(filled, slot_g // k, 0)], -1)
+        slot = np.where(filled, slot_g - base[np.where(filled, src, 0)] * k, -1)
+        out.append((ri[a:b].copy(), rw[a:b].copy(), src.astype(np.int32), slot.astype(np.int32)))
+    return out

@@ -152,3 +152,26 @@ def test_combine_backward_by_enumeration():
             assert abs(gw[s][t, j] - dot) <= 1e-12 * (1 + abs(dot))
     for s, idx in enumerate(idx_list):
         assert (gw[s][idx < 0] == 0).all()
+
+
+def test_dispatch_topk_by_enumeration():
+    """Every owner row's expert, weight, source rank and source slot are those
+    of the (source rank, token, slot) the brute-force enumeration puts there;
+    padding rows carry -1 / 0 / -1 / -1."""
+    rng = np.random.default_rng(33)
+    W_, E, k = 3, 9, 3
+    idx_list = [random_ids(rng, T, k, E, unused=0.2, dup=0.2) for T in (5, 0, 7)]
+    w_list = [rng.random(i.shape).astype(np.float32) for i in idx_list]
+    _, RL = MR.layout(idx_list, E, W_, 2)
+    got = MR.dispatch_topk(RL, idx_list, w_list)
+    want = brute_rows(idx_list, E, W_, 2)
+    for r in range(W_):
+        ri, rw, rsrc, rslot = got[r]
+        assert len(ri) == len(want[r])
+        for row, who in enumerate(want[r]):
+            if who is None:
+                assert (ri[row], rw[row], rsrc[row], rslot[row]) == (-1, 0.0, -1, -1)
+                continue
+            s, t, j = who
+            assert ri[row] == idx_list[s][t, j] and rw[row] == w_list[s][t, j]
+            assert rsrc[row] == s and rslot[row] == t * k + j
