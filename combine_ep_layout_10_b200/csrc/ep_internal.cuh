@@ -329,6 +329,19 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t *tota
     return excl;
 }
 
+struct RecvTopkPeerArgs {
+    const int2 *dst;           // [T, k] plan: (owner rank, row) of each local slot
+    const int32_t *topk_idx;   // [T, k]
+    const float *w;            // [T, k] or nullptr
+    int T, k, rank, epr, capacity;
+    int32_t *const *p_idx;     // [world] per-row expert id tables, or nullptr
+    float *const *p_w;         // [world] per-row weight tables, or nullptr
+    int32_t *const *p_src;     // [world] per-row source rank tables, or nullptr
+    int32_t *const *p_slot;    // [world] per-row source slot tables, or nullptr
+    const int32_t *recv_seg;   // [epr + 1] this rank's segments (plan)
+    const int32_t *recv_cnt;   // [epr] this rank's per-expert slot counts (plan)
+};
+
 struct PlanArgs {
     const int32_t *topk_idx;   // [T, k] this rank's ids
     const int32_t *pos;        // [T, k] local layout (packed, alignment 1)
@@ -373,6 +386,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
 cudaError_t launch_recv_topk(const RecvTopkArgs &a, cudaStream_t s);
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
+cudaError_t launch_recv_topk_peer(const RecvTopkPeerArgs &a, cudaStream_t s);
 // Peer-addressed variants of dispatch and combine (DispatchArgs::dst, CombineArgs::src).
 cudaError_t launch_dispatch_peer(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine_peer(const CombineArgs &a, cudaStream_t s);

@@ -153,6 +153,11 @@ struct ep_peers {
     float *const *recv_scales;   // [world] or nullptr
     const uint8_t *const *y;     // [world] or nullptr
     uint8_t *const *grad_y;      // [world] or nullptr
+    void *topk_block;            // device copy of the per-row output tables (ep_peers_set_topk)
+    int32_t *const *topk_idx;    // [world] or nullptr
+    float *const *topk_w;        // [world] or nullptr
+    int32_t *const *topk_src;    // [world] or nullptr
+    int32_t *const *topk_slot;   // [world] or nullptr
 };
 
 extern "C" {
@@ -209,7 +214,72 @@ ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_sca
 void ep_peers_free(ep_peers *p) {
     if (p == nullptr) return;
     if (p->block) cudaFree(p->block);
+    if (p->topk_block) cudaFree(p->topk_block);
     delete p;
+}
+
+ep_status ep_peers_set_topk(ep_peers *p, int32_t *const *recv_topk_idx, float *const *recv_topk_weights,
+                            int32_t *const *recv_src_rank, int32_t *const *recv_slot) {
+    if (p == nullptr) return EP_ERR_INVALID_ARG;
+    const void *const *tabs[4] = {reinterpret_cast<const void *const *>(recv_topk_idx),
+                                  reinterpret_cast<const void *const *>(recv_topk_weights),
+                                  reinterpret_cast<const void *const *>(recv_src_rank),
+                                  reinterpret_cast<const void *const *>(recv_slot)};
+    for (const void *const *t : tabs)
+        if (t != nullptr)
+            for (int r = 0; r < p->world; ++r)
+                if (t[r] == nullptr || !aligned(t[r], 4)) return EP_ERR_INVALID_ARG;
+    const size_t n = (size_t)p->world;
+    uintptr_t *host = static_cast<uintptr_t *>(std::malloc(4 * n * sizeof(uintptr_t)));
+    if (host == nullptr) return EP_ERR_OOM;
+    for (int i = 0; i < 4; ++i)
+        for (size_t r = 0; r < n; ++r) host[i * n + r] = tabs[i] ? reinterpret_cast<uintptr_t>(tabs[i][r]) : 0;
+    void *block = nullptr;
+    cudaError_t e = cudaMalloc(&block, 4 * n * sizeof(uintptr_t));
+    if (e == cudaSuccess) e = cudaMemcpy(block, host, 4 * n * sizeof(uintptr_t), cudaMemcpyHostToDevice);
+    std::free(host);
+    if (e != cudaSuccess) {
+        if (block) cudaFree(block);
+        return cuda_status(e);
+    }
+    if (p->topk_block) cudaFree(p->topk_block);
+    p->topk_block = block;
+    uintptr_t *tab = static_cast<uintptr_t *>(block);
+    p->topk_idx = recv_topk_idx ? reinterpret_cast<int32_t *const *>(tab) : nullptr;
+    p->topk_w = recv_topk_weights ? reinterpret_cast<float *const *>(tab + n) : nullptr;
+    p->topk_src = recv_src_rank ? reinterpret_cast<int32_t *const *>(tab + 2 * n) : nullptr;
+    p->topk_slot = recv_slot ? reinterpret_cast<int32_t *const *>(tab + 3 * n) : nullptr;
+    return EP_OK;
+}
+
+ep_status ep_dispatch_topk_peer(const ep_plan *plan, const ep_peers *peers, const int32_t *topk_idx,
+                                const float *topk_w, ep_stream_t stream) {
+    if (plan == nullptr || peers == nullptr || peers->world != plan->world) return EP_ERR_INVALID_ARG;
+    if (peers->recv_rows < (size_t)plan->recv_rows) return EP_ERR_INVALID_ARG;
+    if (peers->topk_idx == nullptr && peers->topk_w == nullptr && peers->topk_src == nullptr &&
+        peers->topk_slot == nullptr)
+        return EP_ERR_INVALID_ARG;  // no tables registered (ep_peers_set_topk)
+    if (plan->T > 0) {
+        if (topk_idx == nullptr || !aligned(topk_idx, 4)) return EP_ERR_INVALID_ARG;
+        if (peers->topk_w != nullptr && (topk_w == nullptr || !aligned(topk_w, 4))) return EP_ERR_INVALID_ARG;
+    }
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != plan->device || dev != peers->device) return EP_ERR_INVALID_ARG;
+    RecvTopkPeerArgs a{};
+    a.dst = plan->dst;
+    a.topk_idx = topk_idx;
+    a.w = topk_w;
+    a.T = plan->T; a.k = plan->k; a.rank = plan->rank; a.epr = plan->epr; a.capacity = plan->capacity;
+    a.p_idx = peers->topk_idx;
+    a.p_w = peers->topk_w;
+    a.p_src = peers->topk_src;
+    a.p_slot = peers->topk_slot;
+    a.recv_seg = plan->recv_seg;
+    a.recv_cnt = plan->recv_cnt;
+    return cuda_status(launch_recv_topk_peer(a, stream));
 }
 
 ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const void *x, const float *x_scales,

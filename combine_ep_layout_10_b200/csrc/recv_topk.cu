@@ -97,7 +97,58 @@ __global__ void __launch_bounds__(kTopkThreads) recv_topk_kernel(RecvTopkArgs a)
     if (a.out_slot != nullptr) a.out_slot[r] = s_out;
 }
 
+// Across GPUs (ep_dispatch_topk_peer): every source rank writes, for each of
+// its slots, the expert id, the weight, its rank and the slot's flat index
+// into the owner's per-row tables at the plan's (rank, row); and every rank
+// fills its own padding rows (which no source writes) with -1, 0, -1, -1,
+// so the two parts need no ordering between them.
+constexpr int kTopkPeerThreads = 256;
+
+__global__ void __launch_bounds__(kTopkPeerThreads) recv_topk_peer_scatter_kernel(RecvTopkPeerArgs a) {
+    pdl_wait_then_trigger();
+    const int64_t s = (int64_t)blockIdx.x * kTopkPeerThreads + threadIdx.x;
+    if (s >= (int64_t)a.T * a.k) return;
+    const int2 d = __ldg(a.dst + s);
+    if (d.x < 0) return;
+    if (a.p_idx != nullptr) a.p_idx[d.x][d.y] = __ldg(a.topk_idx + s);
+    if (a.p_w != nullptr) a.p_w[d.x][d.y] = a.w != nullptr ? __ldg(a.w + s) : 0.0f;
+    if (a.p_src != nullptr) a.p_src[d.x][d.y] = a.rank;
+    if (a.p_slot != nullptr) a.p_slot[d.x][d.y] = (int32_t)s;
+}
+
+__global__ void __launch_bounds__(kTopkPeerThreads) recv_topk_peer_pad_kernel(RecvTopkPeerArgs a) {
+    pdl_wait_then_trigger();
+    const int lane = threadIdx.x & 31;
+    const int le = blockIdx.x * (kTopkPeerThreads / 32) + (threadIdx.x >> 5);  // this rank's expert
+    if (le >= a.epr) return;
+    int32_t used = __ldg(a.recv_cnt + le);
+    if (a.capacity > 0 && used > a.capacity) used = a.capacity;
+    const int64_t start = (int64_t)__ldg(a.recv_seg + le) + used;
+    const int64_t end = __ldg(a.recv_seg + le + 1);
+    int32_t *idx = a.p_idx != nullptr ? a.p_idx[a.rank] : nullptr;
+    float *w = a.p_w != nullptr ? a.p_w[a.rank] : nullptr;
+    int32_t *src = a.p_src != nullptr ? a.p_src[a.rank] : nullptr;
+    int32_t *slot = a.p_slot != nullptr ? a.p_slot[a.rank] : nullptr;
+    for (int64_t row = start + lane; row < end; row += 32) {
+        if (idx != nullptr) idx[row] = -1;
+        if (w != nullptr) w[row] = 0.0f;
+        if (src != nullptr) src[row] = -1;
+        if (slot != nullptr) slot[row] = -1;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_recv_topk_peer(const RecvTopkPeerArgs &a, cudaStream_t s) {
+    const int64_t slots = (int64_t)a.T * a.k;
+    cudaError_t e = cudaSuccess;
+    if (slots > 0)
+        e = launch_kernel(recv_topk_peer_scatter_kernel, (unsigned)((slots + kTopkPeerThreads - 1) / kTopkPeerThreads),
+                          kTopkPeerThreads, 0, s, a);
+    if (e != cudaSuccess || a.epr == 0) return e;
+    const int per_block = kTopkPeerThreads / 32;
+    return launch_kernel(recv_topk_peer_pad_kernel, (a.epr + per_block - 1) / per_block, kTopkPeerThreads, 0, s, a);
+}
 
 cudaError_t launch_recv_topk(const RecvTopkArgs &a, cudaStream_t s) {
     if (a.n_rows == 0) return cudaSuccess;

@@ -45,7 +45,7 @@ ABI_SYMBOLS = (
     "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk",
     "ep_peer_max_recv_rows", "ep_plan_create", "ep_plan_free", "ep_plan_export", "ep_plan_recv_rows_host",
     "ep_plan_check", "ep_peers_create", "ep_peers_free", "ep_dispatch_peer", "ep_combine_peer",
-    "ep_combine_backward_peer",
+    "ep_combine_backward_peer", "ep_peers_set_topk", "ep_dispatch_topk_peer",
     "ep_ipc_export", "ep_ipc_import", "ep_ipc_release",
 )
 
@@ -136,6 +136,10 @@ def lib() -> ctypes.CDLL:
         L.ep_combine_peer.restype = I
         L.ep_combine_backward_peer.argtypes = [P, P, P, P, I, P, P]
         L.ep_combine_backward_peer.restype = I
+        L.ep_peers_set_topk.argtypes = [P, P, P, P, P]
+        L.ep_peers_set_topk.restype = I
+        L.ep_dispatch_topk_peer.argtypes = [P, P, P, P, P]
+        L.ep_dispatch_topk_peer.restype = I
         L.ep_ipc_export.argtypes = [P, P, ctypes.POINTER(U64)]
         L.ep_ipc_export.restype = I
         L.ep_ipc_import.argtypes = [P, U64, ctypes.POINTER(P)]
@@ -549,6 +553,13 @@ class Peers:
             raise RuntimeError("peer table already freed")
         return self._ptr
 
+    def set_topk(self, recv_topk_idx=None, recv_topk_weights=None, recv_src_rank=None, recv_slot=None):
+        """Register every rank's per-row output tables (lists of `world`
+        tensors or device addresses, each [recv_rows])."""
+        arrs = [_ptr_array(t) if t is not None else None
+                for t in (recv_topk_idx, recv_topk_weights, recv_src_rank, recv_slot)]
+        _check(lib().ep_peers_set_topk(self.ptr, *arrs), "ep_peers_set_topk")
+
     def free(self) -> None:
         if self._ptr is not None:
             lib().ep_peers_free(self._ptr)
@@ -609,6 +620,18 @@ def ep_combine_backward_peer(plan: Plan, peers: Peers, grad_out: torch.Tensor, t
                                                     (plan.num_tokens, plan.num_topk)), _stream(stream))
     _check(st, "ep_combine_backward_peer")
     return grad_weights
+
+
+def ep_dispatch_topk_peer(plan: Plan, peers: Peers, topk_idx: torch.Tensor,
+                          topk_weights: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Writes every local slot's expert id, weight, rank and slot index into
+    its owner's per-row tables (Peers.set_topk) and fills this rank's own
+    padding rows with -1 / 0 / -1 / -1."""
+    st = lib().ep_dispatch_topk_peer(plan.ptr, peers.ptr,
+                                     _dev_ptr(topk_idx, torch.int32, "topk_idx", (plan.num_tokens, plan.num_topk)),
+                                     _dev_ptr(topk_weights, torch.float32, "topk_weights",
+                                              (plan.num_tokens, plan.num_topk)), _stream(stream))
+    _check(st, "ep_dispatch_topk_peer")
 
 
 def ipc_export(t: torch.Tensor):

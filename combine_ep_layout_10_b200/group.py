@@ -56,13 +56,19 @@ class EpGroup:
         self.recv_scales = torch.empty(recv_rows, hidden // 128, dtype=torch.float32, device=dev) if fp8 else None
         self.y = torch.empty(recv_rows, hidden, dtype=torch.bfloat16, device=dev)
         self.grad_y = torch.empty(recv_rows, hidden, dtype=torch.bfloat16, device=dev)
-        mine = [self.recv_x, self.recv_scales, self.y, self.grad_y]
+        # per-row routing outputs of each received row: expert, weight, source rank, source slot
+        self.recv_topk_idx = torch.empty(recv_rows, dtype=torch.int32, device=dev)
+        self.recv_topk_weights = torch.empty(recv_rows, dtype=torch.float32, device=dev)
+        self.recv_src_rank = torch.empty(recv_rows, dtype=torch.int32, device=dev)
+        self.recv_slot = torch.empty(recv_rows, dtype=torch.int32, device=dev)
+        mine = [self.recv_x, self.recv_scales, self.y, self.grad_y,
+                self.recv_topk_idx, self.recv_topk_weights, self.recv_src_rank, self.recv_slot]
         handles = [ep.ipc_export(t) if t is not None else None for t in mine]
         torch.cuda.synchronize(dev)
         everyone = [None] * self.world
         dist.all_gather_object(everyone, handles, group=group)
         self._imported = []   # (address, offset) to release
-        tables = [[], [], [], []]
+        tables = [[] for _ in mine]
         for r in range(self.world):
             for i, t in enumerate(mine):
                 if t is None:
@@ -76,6 +82,7 @@ class EpGroup:
                     tables[i].append(addr)
         self.peers = ep.Peers(self.world, tables[0], tables[1] if fp8 else None, tables[2], recv_rows,
                               grad_y=tables[3])
+        self.peers.set_topk(*tables[4:8])
 
     # -- collectives -------------------------------------------------------
 
@@ -109,10 +116,13 @@ class EpGroup:
 
     def dispatch(self, x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
                  plan: Optional[ep.Plan] = None, expert_alignment: int = 1, capacity: int = 0,
-                 x_scales: Optional[torch.Tensor] = None, num_sms: int = 0) -> ep.Plan:
+                 x_scales: Optional[torch.Tensor] = None, num_sms: int = 0,
+                 topk_weights: Optional[torch.Tensor] = None) -> ep.Plan:
         """Sends this rank's tokens to their experts' owners.  Pass `plan` (a
         cached handle) when the routing has not changed.  On return, in stream
-        order, this rank's receive buffer holds its rows from every rank."""
+        order, this rank's receive buffer holds its rows from every rank; with
+        `topk_weights` (and `topk_idx`) recv_topk_idx / recv_topk_weights /
+        recv_src_rank / recv_slot also describe every received row."""
         if plan is None:
             if topk_idx is None:
                 raise ValueError("dispatch needs topk_idx or a plan")
@@ -120,6 +130,10 @@ class EpGroup:
         else:
             self._barrier()   # peers have finished reading the previous step
         ep.ep_dispatch_peer(plan, self.peers, x, self.fp8, x_scales=x_scales, num_sms=num_sms)
+        if topk_weights is not None:
+            if topk_idx is None:
+                raise ValueError("per-row outputs need topk_idx")
+            ep.ep_dispatch_topk_peer(plan, self.peers, topk_idx, topk_weights)
         self._barrier()       # every rank's stores are complete
         return plan
 

@@ -408,6 +408,26 @@ ep_status ep_peers_create(int world, void *const *recv_x, float *const *recv_sca
                           void *const *grad_y, size_t recv_rows, ep_peers **out);
 void ep_peers_free(ep_peers *peers);
 
+/* Per-row routing output tables of every rank (host arrays of `world`
+ * device pointers, each [recv_rows], 4-byte aligned; any array may be NULL):
+ * the expert id, the routing weight, the source rank and the source slot
+ * (t * k + j on that rank) of each receive row.  Copied to device memory the
+ * peer table owns; a second call replaces the first. */
+ep_status ep_peers_set_topk(ep_peers *peers, int32_t *const *recv_topk_idx, float *const *recv_topk_weights,
+                            int32_t *const *recv_src_rank, int32_t *const *recv_slot);
+
+/* Per-row routing outputs across ranks: the pages' recv_topk_idx and
+ * recv_topk_weights on the receiving side (docsearch item 10).  Every local
+ * slot (t, j) with a row writes topk_idx[t][j], topk_weights[t][j], this
+ * rank and t * k + j into the owner's tables at that row; this rank's own
+ * rows that no slot fills (alignment or capacity padding inside its
+ * received rows) get -1, 0.0f, -1, -1.  Rows past the received ones are not
+ * touched.  topk_idx: device int32 [T, k] (the ids the plan was made from);
+ * topk_weights: device fp32 [T, k], needed when a weight table is set.
+ * Ordered like ep_dispatch_peer (the caller's collectives). */
+ep_status ep_dispatch_topk_peer(const ep_plan *plan, const ep_peers *peers, const int32_t *topk_idx,
+                                const float *topk_weights, ep_stream_t stream);
+
 /* Dispatch across ranks: as ep_dispatch_ex, with row (d.y) of rank d.x's
  * buffers as the destination of each slot (d from the plan), written with
  * plain 16-byte stores through the peer mappings; scales row-major.  The

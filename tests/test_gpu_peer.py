@@ -306,3 +306,36 @@ def test_metric_batch_over_eight_ranks_sampled():
             want = oracle.combine(torch.stack(rows), w_list[s][t:t + 1].numpy(),
                                   np.arange(base.k, dtype=np.int32)[None, :])
             assert (u16(outs[s][t:t + 1]) == want).all()
+
+
+@pytest.mark.parametrize("name,Ts,align,cap", [("tiny", [40, 0, 17, 64], 4, 0),
+                                               ("prefill", [64, 30, 0, 100], 1, 0),
+                                               ("decode", [128] * 8, 1, 128)])
+def test_peer_dispatch_topk(name, Ts, align, cap):
+    """Per-row outputs on the owners: expert, weight, source rank and slot of
+    every received row exactly the oracle's; padding rows -1 / 0 / -1 / -1;
+    rows past the received ones untouched."""
+    base, idx_list, _, w_list = routing(name, Ts, unused=True, H=512 if name == "decode" else None)
+    Wr = len(Ts)
+    em = Emulated(base.E, base.k, base.H, idx_list, False, align, cap)
+    rows = em.recv_rows
+    t_idx = [torch.full((rows,), -7, dtype=torch.int32, device=DEV) for _ in range(Wr)]
+    t_w = [torch.full((rows,), -7.0, dtype=torch.float32, device=DEV) for _ in range(Wr)]
+    t_src = [torch.full((rows,), -7, dtype=torch.int32, device=DEV) for _ in range(Wr)]
+    t_slot = [torch.full((rows,), -7, dtype=torch.int32, device=DEV) for _ in range(Wr)]
+    em.peers.set_topk(t_idx, t_w, t_src, t_slot)
+    for r in range(Wr):
+        ep.ep_dispatch_topk_peer(em.plans[r], em.peers, em.idx_dev[r], w_list[r].to(DEV))
+    torch.cuda.synchronize()
+    _, RL = MR.layout(idx_list, base.E, Wr, align, cap)
+    want = MR.dispatch_topk(RL, idx_list, w_list)
+    for r in range(Wr):
+        n = RL.recv_rows(r)
+        wi, ww, ws, wsl = want[r]
+        assert (t_idx[r][:n].cpu().numpy() == wi).all()
+        assert (t_w[r][:n].cpu().numpy().view(np.uint32) == ww.view(np.uint32)).all()
+        assert (t_src[r][:n].cpu().numpy() == ws).all()
+        assert (t_slot[r][:n].cpu().numpy() == wsl).all()
+        for t in (t_idx, t_src, t_slot):
+            assert (t[r][n:].cpu().numpy() == -7).all()
+        assert (t_w[r][n:].cpu().numpy() == -7.0).all()

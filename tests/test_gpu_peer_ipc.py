@@ -65,9 +65,14 @@ def _worker(rank, world, port, q, backend="gloo"):
             return bool((got_q[filled] == q_want[filled]).all()
                         and (got_s[filled].view(np.uint32) == s_want[filled].view(np.uint32)).all())
 
-        plan = g.dispatch(x_list[rank].cuda(), idx_list[rank].cuda())
+        plan = g.dispatch(x_list[rank].cuda(), idx_list[rank].cuda(), topk_weights=w_list[rank].cuda())
         torch.cuda.synchronize()
         result["dispatch"] = check_recv(x_list)
+        wi, ww, wsrc, wslot = MR.dispatch_topk(RL, idx_list, w_list)[rank]
+        result["topk"] = bool((g.recv_topk_idx[:n].cpu().numpy() == wi).all()
+                              and (g.recv_topk_weights[:n].cpu().numpy().view(np.uint32) == ww.view(np.uint32)).all()
+                              and (g.recv_src_rank[:n].cpu().numpy() == wsrc).all()
+                              and (g.recv_slot[:n].cpu().numpy() == wslot).all())
         result["rows"] = plan.recv_rows_host() == n
         ys = [W.make_expert_out(recv_rows, H, seed=900 + r) for r in range(world)]
         g.y.copy_(ys[rank].cuda())
@@ -128,7 +133,7 @@ def _run(world, backend):
     for r in sorted(results, key=lambda d: d["rank"]):
         assert r["error"] is None, r
         assert r["dispatch"] and r["rows"] and r["combine"] and r["cached"], r
-        assert r["combine_bwd"] and r["dispatch_bwd"], r
+        assert r["combine_bwd"] and r["dispatch_bwd"] and r["topk"], r
 
 
 def test_two_processes_share_buffers_over_ipc():
