@@ -283,7 +283,8 @@ ep_status ep_dispatch_topk_peer(const ep_plan *plan, const ep_peers *peers, cons
 }
 
 ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const void *x, const float *x_scales,
-                           int H, int in_format, int out_format, int num_sms, ep_stream_t stream) {
+                           int H, int in_format, int out_format, int64_t scale_row_stride,
+                           int64_t scale_group_stride, int num_sms, ep_stream_t stream) {
     if (plan == nullptr || peers == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
     if (peers->world != plan->world || peers->recv_rows < (size_t)plan->recv_rows) return EP_ERR_INVALID_ARG;
     const bool in_fp8 = in_format == EP_FORMAT_E4M3;
@@ -292,6 +293,13 @@ ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const voi
         return EP_ERR_INVALID_ARG;
     if (in_fp8 && !out_fp8) return EP_ERR_INVALID_ARG;
     if (out_fp8 && (H % 128 != 0 || peers->recv_scales == nullptr)) return EP_ERR_INVALID_ARG;
+    if (out_fp8) {
+        // Non-overlapping scale layouts only, as ep_dispatch_ex: row-major-like or column-major-like.
+        const int64_t G = H / 128;
+        const bool row_like = scale_group_stride == 1 && scale_row_stride >= G;
+        const bool col_like = scale_row_stride == 1 && scale_group_stride >= (int64_t)peers->recv_rows;
+        if (!(row_like || col_like)) return EP_ERR_INVALID_ARG;
+    }
     if (plan->T > 0) {
         if (x == nullptr || !aligned(x, 16)) return EP_ERR_INVALID_ARG;
         if (in_fp8 && (x_scales == nullptr || !aligned(x_scales, 4))) return EP_ERR_INVALID_ARG;
@@ -310,8 +318,8 @@ ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const voi
     a.dst = plan->dst;
     a.peer_recv = peers->recv_x;
     a.peer_scales = out_fp8 ? peers->recv_scales : nullptr;
-    a.s_row = H / 128;
-    a.s_grp = 1;
+    a.s_row = scale_row_stride;
+    a.s_grp = scale_group_stride;
     a.mode = !out_fp8 ? kDispatchCopyBf16 : in_fp8 ? kDispatchCopyFp8 : kDispatchQuantFp8;
     a.num_sms = num_sms;
     a.T = plan->T; a.k = plan->k; a.H = H;

@@ -130,7 +130,7 @@ def lib() -> ctypes.CDLL:
         L.ep_peers_create.restype = I
         L.ep_peers_free.argtypes = [P]
         L.ep_peers_free.restype = None
-        L.ep_dispatch_peer.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.ep_dispatch_peer.argtypes = [P, P, P, P, I, I, I, I64, I64, I, P]
         L.ep_dispatch_peer.restype = I
         L.ep_combine_peer.argtypes = [P, P, P, I, P, I, P]
         L.ep_combine_peer.restype = I
@@ -573,17 +573,27 @@ class Peers:
 
 
 def ep_dispatch_peer(plan: Plan, peers: Peers, x: torch.Tensor, use_fp8: bool,
-                     x_scales: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None) -> None:
+                     x_scales: Optional[torch.Tensor] = None, num_sms: int = 0,
+                     scale_layout: str = "row", scale_ld: Optional[int] = None, stream=None) -> None:
     """Stores every local token's rows (BF16, fused FP8, or pre-quantised FP8
-    when x is float8_e4m3fn with x_scales) into the owners' receive buffers."""
+    when x is float8_e4m3fn with x_scales) into the owners' receive buffers;
+    scales row-major [rows, H/128] or column-major [H/128, scale_ld]
+    (scale_ld >= the peer table's recv_rows, default recv_rows)."""
     T, H = x.shape
     in_fp8 = x.dtype == torch.float8_e4m3fn
     if in_fp8 and not use_fp8:
         raise ValueError("FP8 input needs FP8 output")
+    if scale_layout == "row":
+        s_row, s_grp = H // 128, 1
+    elif scale_layout == "col":
+        s_row, s_grp = 1, scale_ld if scale_ld is not None else peers.recv_rows
+    else:
+        raise ValueError("scale_layout must be 'row' or 'col'")
     st = lib().ep_dispatch_peer(plan.ptr, peers.ptr, _dev_ptr(x, x.dtype, "x", (plan.num_tokens, H)),
                                 _dev_ptr(x_scales, torch.float32, "x_scales"), H,
                                 EP_FORMAT_E4M3 if in_fp8 else EP_FORMAT_BF16,
-                                EP_FORMAT_E4M3 if use_fp8 else EP_FORMAT_BF16, num_sms, _stream(stream))
+                                EP_FORMAT_E4M3 if use_fp8 else EP_FORMAT_BF16, s_row, s_grp, num_sms,
+                                _stream(stream))
     _check(st, "ep_dispatch_peer")
 
 

@@ -430,10 +430,15 @@ ep_status ep_dispatch_topk_peer(const ep_plan *plan, const ep_peers *peers, cons
 
 /* Dispatch across ranks: as ep_dispatch_ex, with row (d.y) of rank d.x's
  * buffers as the destination of each slot (d from the plan), written with
- * plain 16-byte stores through the peer mappings; scales row-major.  The
- * caller orders these stores before the owners' reads with a collective. */
+ * plain 16-byte stores through the peer mappings.  Scales of row p and group
+ * g go to recv_scales[p * scale_row_stride + g * scale_group_stride] in the
+ * owner's buffer, row-major (group stride 1, row stride >= H/128) or
+ * column-major (row stride 1, group stride >= the peer table's recv_rows);
+ * every rank's scale buffer must hold that layout.  The caller orders these
+ * stores before the owners' reads with a collective. */
 ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const void *x, const float *x_scales,
-                           int hidden, int in_format, int out_format, int num_sms, ep_stream_t stream);
+                           int hidden, int in_format, int out_format, int64_t scale_row_stride,
+                           int64_t scale_group_stride, int num_sms, ep_stream_t stream);
 
 /* Combine across ranks: as ep_combine_ex, reading each slot's expert-output
  * row from its owner's y buffer through the peer mappings.  topk_weights

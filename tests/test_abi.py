@@ -110,7 +110,7 @@ def test_multi_gpu_argument_errors_on_host(L):
     nul = (P * 2)(256, None)
     assert L.ep_peers_create(2, nul, None, None, None, 64, ctypes.byref(out)) == INV
     # peer calls with no plan or table
-    assert L.ep_dispatch_peer(None, None, fake, None, 128, 0, 1, 0, None) == INV
+    assert L.ep_dispatch_peer(None, None, fake, None, 128, 0, 1, 1, 1, 0, None) == INV
     assert L.ep_combine_peer(None, None, None, 128, fake, 0, None) == INV
     assert L.ep_combine_backward_peer(None, None, fake, fake, 128, None, None) == INV
     # IPC: null arguments

@@ -339,3 +339,31 @@ def test_peer_dispatch_topk(name, Ts, align, cap):
         for t in (t_idx, t_src, t_slot):
             assert (t[r][n:].cpu().numpy() == -7).all()
         assert (t_w[r][n:].cpu().numpy() == -7.0).all()
+
+
+def test_peer_dispatch_column_major_scales():
+    """FP8 scales written column-major ([H/128, ld] per owner, the FP8 grouped
+    GEMM layout) hold exactly the row-major scales, transposed; padding
+    columns and the columns past the received rows stay untouched."""
+    base, idx_list, x_list, _ = routing("prefill", [100, 0, 57, 31])
+    Wr, H = 4, base.H
+    em = Emulated(base.E, base.k, H, idx_list, True)
+    rows = em.recv_rows
+    ld = (rows + 3) // 4 * 4
+    cols = [torch.full((H // 128, ld), -3.0, dtype=torch.float32, device=DEV) for _ in range(Wr)]
+    peers = ep.Peers(Wr, em.recv, cols, None, rows)
+    for r in range(Wr):
+        ep.ep_dispatch_peer(em.plans[r], peers, x_list[r].to(DEV), True, scale_layout="col", scale_ld=ld)
+    torch.cuda.synchronize()
+    _, RL = MR.layout(idx_list, base.E, Wr)
+    want = MR.dispatch_fp8(RL, x_list)
+    for r in range(Wr):
+        n = RL.recv_rows(r)
+        f = filled_rows(RL, r)
+        got = cols[r].cpu().numpy()
+        assert (got[:, :n].T[f].view(np.uint32) == want[r][1][f].view(np.uint32)).all()
+        assert (got[:, :n].T[~f] == -3.0).all() and (got[:, n:] == -3.0).all()
+        assert (em.recv[r][:n].cpu().numpy()[f] == want[r][0][f]).all()
+    # a scale layout that would overlap is refused on the host
+    with pytest.raises(ep.EpError):
+        ep.ep_dispatch_peer(em.plans[0], peers, x_list[0].to(DEV), True, scale_layout="col", scale_ld=ld - 8)
