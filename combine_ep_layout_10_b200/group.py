@@ -38,10 +38,13 @@ class EpGroup:
     recv_rows: rows of every rank's receive buffer (the same on all ranks);
     ep.ep_peer_max_recv_rows() gives a bound that always suffices.
     fp8: receive buffers hold e4m3 codes + fp32 scales (else bf16).
+    scale_layout: "row" (scales [recv_rows, H/128]) or "col" ([H/128, ld],
+    ld = recv_rows rounded up to 4: the FP8 grouped-GEMM layout).
     """
 
     def __init__(self, num_experts: int, hidden: int, recv_rows: int, fp8: bool = True,
-                 group: Optional[dist.ProcessGroup] = None, device: Optional[torch.device] = None):
+                 group: Optional[dist.ProcessGroup] = None, device: Optional[torch.device] = None,
+                 scale_layout: str = "row"):
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
@@ -53,7 +56,16 @@ class EpGroup:
         dev = self.device
         self.recv_x = torch.empty(recv_rows, hidden, dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16,
                                   device=dev)
-        self.recv_scales = torch.empty(recv_rows, hidden // 128, dtype=torch.float32, device=dev) if fp8 else None
+        if scale_layout not in ("row", "col"):
+            raise ValueError("scale_layout must be 'row' or 'col'")
+        self.scale_layout = scale_layout
+        self.scale_ld = (recv_rows + 3) // 4 * 4
+        if not fp8:
+            self.recv_scales = None
+        elif scale_layout == "row":
+            self.recv_scales = torch.empty(recv_rows, hidden // 128, dtype=torch.float32, device=dev)
+        else:
+            self.recv_scales = torch.empty(hidden // 128, self.scale_ld, dtype=torch.float32, device=dev)
         self.y = torch.empty(recv_rows, hidden, dtype=torch.bfloat16, device=dev)
         self.grad_y = torch.empty(recv_rows, hidden, dtype=torch.bfloat16, device=dev)
         # per-row routing outputs of each received row: expert, weight, source rank, source slot
@@ -129,7 +141,8 @@ class EpGroup:
             plan = self.make_plan(topk_idx, expert_alignment, capacity)   # its all-gather orders our stores
         else:
             self._barrier()   # peers have finished reading the previous step
-        ep.ep_dispatch_peer(plan, self.peers, x, self.fp8, x_scales=x_scales, num_sms=num_sms)
+        ep.ep_dispatch_peer(plan, self.peers, x, self.fp8, x_scales=x_scales, num_sms=num_sms,
+                            scale_layout=self.scale_layout, scale_ld=self.scale_ld)
         if topk_weights is not None:
             if topk_idx is None:
                 raise ValueError("per-row outputs need topk_idx")

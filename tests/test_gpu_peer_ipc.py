@@ -29,7 +29,7 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q, backend="gloo"):
+def _worker(rank, world, port, q, backend="gloo", scale_layout="row"):
     import sys
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -53,7 +53,7 @@ def _worker(rank, world, port, q, backend="gloo"):
         idx_list = [r[1] for r in routed]
         w_list = [r[2] for r in routed]
         recv_rows = ep.ep_peer_max_recv_rows(sum(tokens), k, E, world)
-        g = group.EpGroup(E, H, recv_rows, fp8=True)
+        g = group.EpGroup(E, H, recv_rows, fp8=True, scale_layout=scale_layout)
         _, RL = MR.layout(idx_list, E, world)
         n = RL.recv_rows(rank)
         filled = RL.L.src_idx[RL.L.rank_off[rank]:RL.L.rank_off[rank] + n] >= 0
@@ -61,7 +61,7 @@ def _worker(rank, world, port, q, backend="gloo"):
         def check_recv(xs):
             q_want, s_want = MR.dispatch_fp8(RL, xs)[rank]
             got_q = g.recv_x[:n].view(torch.uint8).cpu().numpy()
-            got_s = g.recv_scales[:n].cpu().numpy()
+            got_s = (g.recv_scales[:n] if scale_layout == "row" else g.recv_scales[:, :n].T).cpu().numpy()
             return bool((got_q[filled] == q_want[filled]).all()
                         and (got_s[filled].view(np.uint32) == s_want[filled].view(np.uint32)).all())
 
@@ -110,7 +110,7 @@ def _worker(rank, world, port, q, backend="gloo"):
         dist.destroy_process_group()
 
 
-def _run(world, backend):
+def _run(world, backend, scale_layout="row"):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     from combine_ep_layout_10_b200 import build
@@ -118,7 +118,7 @@ def _run(world, backend):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q, backend)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, backend, scale_layout)) for r in range(world)]
     for p in procs:
         p.start()
     results = []
@@ -143,5 +143,5 @@ def test_two_processes_share_buffers_over_ipc():
 def test_single_rank_group_over_nccl():
     """The NCCL branch of EpGroup (device-ordered all-reduce barriers and the
     all_gather_into_tensor of the counts) with one rank, whose peer table is
-    its own buffers."""
-    _run(1, "nccl")
+    its own buffers; FP8 scales in the column-major (grouped-GEMM) layout."""
+    _run(1, "nccl", "col")
