@@ -367,3 +367,28 @@ def test_peer_dispatch_column_major_scales():
     # a scale layout that would overlap is refused on the host
     with pytest.raises(ep.EpError):
         ep.ep_dispatch_peer(em.plans[0], peers, x_list[0].to(DEV), True, scale_layout="col", scale_ld=ld - 8)
+
+
+@pytest.mark.parametrize("num_sms", [1, 7])
+def test_peer_sm_budget_changes_nothing(num_sms):
+    """The SM budget changes the peer kernels' launch shape, never the result."""
+    base, idx_list, x_list, w_list = routing("group_limited", [300, 128, 77])
+    Wr = 3
+    em = Emulated(base.E, base.k, base.H, idx_list, True)
+    em.dispatch(x_list)
+    ref_q = [r.clone() for r in em.recv]
+    ref_s = [s.clone() for s in em.scales]
+    for r in em.recv:
+        r.fill_(SENTINEL)
+    for r in range(Wr):
+        ep.ep_dispatch_peer(em.plans[r], em.peers, x_list[r].to(DEV), True, num_sms=num_sms)
+    gy = torch.Generator(device=DEV).manual_seed(5)
+    for r in range(Wr):
+        em.y[r].copy_(torch.randn(em.recv_rows, base.H, generator=gy, device=DEV).to(torch.bfloat16))
+    outs0 = [ep.ep_combine_peer(em.plans[r], em.peers, w_list[r].to(DEV), base.H) for r in range(Wr)]
+    outs1 = [ep.ep_combine_peer(em.plans[r], em.peers, w_list[r].to(DEV), base.H, num_sms=num_sms)
+             for r in range(Wr)]
+    torch.cuda.synchronize()
+    for r in range(Wr):
+        assert torch.equal(em.recv[r], ref_q[r]) and torch.equal(em.scales[r], ref_s[r])
+        assert torch.equal(outs0[r].view(torch.int16), outs1[r].view(torch.int16))
