@@ -372,8 +372,8 @@ def test_peer_dispatch_column_major_scales():
 @pytest.mark.parametrize("num_sms", [1, 7])
 def test_peer_sm_budget_changes_nothing(num_sms):
     """The SM budget changes the peer kernels' launch shape, never the result."""
-    base, idx_list, x_list, w_list = routing("group_limited", [300, 128, 77])
-    Wr = 3
+    base, idx_list, x_list, w_list = routing("group_limited", [300, 128, 77, 40])
+    Wr = 4
     em = Emulated(base.E, base.k, base.H, idx_list, True)
     em.dispatch(x_list)
     ref_q = [r.clone() for r in em.recv]
