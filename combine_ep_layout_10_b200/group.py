@@ -79,7 +79,11 @@ class EpGroup:
         torch.cuda.synchronize(dev)
         everyone = [None] * self.world
         dist.all_gather_object(everyone, handles, group=group)
-        self._imported = []   # (address, offset) to release
+        # Several buffers can live in one allocation (the caching allocator
+        # packs small ones together): each distinct handle is opened once and
+        # the buffers are addressed by their offsets inside it.
+        self._imported = []   # base addresses of opened handles, to release
+        opened = {}
         tables = [[] for _ in mine]
         for r in range(self.world):
             for i, t in enumerate(mine):
@@ -87,11 +91,12 @@ class EpGroup:
                     continue
                 if r == self.rank:
                     tables[i].append(t.data_ptr())
-                else:
-                    blob, off = everyone[r][i]
-                    addr = ep.ipc_import(blob, off)
-                    self._imported.append((addr, off))
-                    tables[i].append(addr)
+                    continue
+                blob, off = everyone[r][i]
+                if blob not in opened:
+                    opened[blob] = ep.ipc_import(blob, 0)
+                    self._imported.append(opened[blob])
+                tables[i].append(opened[blob] + off)
         self.peers = ep.Peers(self.world, tables[0], tables[1] if fp8 else None, tables[2], recv_rows,
                               grad_y=tables[3])
         self.peers.set_topk(*tables[4:8])
@@ -183,6 +188,6 @@ class EpGroup:
         torch.cuda.synchronize(self.device)
         self.peers.free()
         self.peers = None
-        for addr, off in self._imported:
-            ep.ipc_release(addr, off)
+        for base in self._imported:
+            ep.ipc_release(base, 0)
         self._imported = []
