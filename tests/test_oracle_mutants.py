@@ -73,6 +73,16 @@ MUTANTS = [
     ("grad_y without the weight",
      "float prod = w[s] * g;", "float prod = g;",
      [(PB.test_combine_backward_vs_autograd, {"name": "tiny"})]),
+    ("pre-quantised scales copied from the next token",
+     "memcpy(scales + (int64_t)p * G, xs + (int64_t)t * G, (size_t)G * sizeof(float));",
+     "memcpy(scales + (int64_t)p * G, xs + (int64_t)(t + 1 < T ? t + 1 : t) * G, (size_t)G * sizeof(float));",
+     [(PD.test_prequant_dispatch_equals_quantise_then_dispatch, {"name": "decode"}),
+      (PD.test_prequant_dispatch_equals_quantise_then_dispatch, {"name": "prefill"})]),
+    ("pre-quantised codes of half a row",
+     "memcpy(recv + (int64_t)p * H, xq + (int64_t)t * H, (size_t)H);",
+     "memcpy(recv + (int64_t)p * H, xq + (int64_t)t * H, (size_t)H / 2);",
+     [(PD.test_prequant_dispatch_equals_quantise_then_dispatch, {"name": "decode"}),
+      (PD.test_prequant_dispatch_equals_quantise_then_dispatch, {"name": "prefill"})]),
     ("per-row weight taken from the neighbouring slot",
      "if (recv_w) recv_w[p] = topk_w[s];",
      "if (recv_w) recv_w[p] = topk_w[s ^ 1];",
