@@ -369,6 +369,17 @@ ep_status ep_dispatch_topk(const ep_handle *h, const float *topk_w, int32_t *rec
     return cuda_status(launch_recv_topk(a, stream));
 }
 
+ep_status ep_e4m3_encode(const float *x, uint8_t *codes, size_t n, ep_stream_t stream) {
+    if (n == 0) return EP_OK;
+    if (x == nullptr || codes == nullptr || !aligned(x, 16) || !aligned(codes, 16)) return EP_ERR_INVALID_ARG;
+    if (n >= ((size_t)1 << 40)) return EP_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    return cuda_status(launch_e4m3_encode(x, codes, (int64_t)n, stream));
+}
+
 void ep_handle_free(ep_handle *h) {
     if (h == nullptr) return;
     if (h->block != nullptr) {

@@ -385,6 +385,7 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
 cudaError_t launch_recv_topk(const RecvTopkArgs &a, cudaStream_t s);
+cudaError_t launch_e4m3_encode(const float *x, uint8_t *out, int64_t n, cudaStream_t s);
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
 cudaError_t launch_recv_topk_peer(const RecvTopkPeerArgs &a, cudaStream_t s);
 // Peer-addressed variants of dispatch and combine (DispatchArgs::dst, CombineArgs::src).

@@ -45,7 +45,7 @@ ABI_SYMBOLS = (
     "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk",
     "ep_peer_max_recv_rows", "ep_plan_create", "ep_plan_free", "ep_plan_export", "ep_plan_recv_rows_host",
     "ep_plan_check", "ep_peers_create", "ep_peers_free", "ep_dispatch_peer", "ep_combine_peer",
-    "ep_combine_backward_peer", "ep_peers_set_topk", "ep_dispatch_topk_peer",
+    "ep_combine_backward_peer", "ep_peers_set_topk", "ep_dispatch_topk_peer", "ep_e4m3_encode",
     "ep_ipc_export", "ep_ipc_import", "ep_ipc_release",
 )
 
@@ -140,6 +140,8 @@ def lib() -> ctypes.CDLL:
         L.ep_peers_set_topk.restype = I
         L.ep_dispatch_topk_peer.argtypes = [P, P, P, P, P]
         L.ep_dispatch_topk_peer.restype = I
+        L.ep_e4m3_encode.argtypes = [P, P, S, P]
+        L.ep_e4m3_encode.restype = I
         L.ep_ipc_export.argtypes = [P, P, ctypes.POINTER(U64)]
         L.ep_ipc_export.restype = I
         L.ep_ipc_import.argtypes = [P, U64, ctypes.POINTER(P)]
@@ -386,6 +388,16 @@ def ep_dispatch_topk(handle: Handle, topk_weights: Optional[torch.Tensor] = None
                                 _dev_ptr(rs, torch.int32, "recv_slot"), rows, _stream(stream))
     _check(st, "ep_dispatch_topk")
     return ri, rw, rs
+
+
+def e4m3_encode(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fp32 -> e4m3 codes (uint8, same shape) with the dispatch's rounding."""
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    st = lib().ep_e4m3_encode(_dev_ptr(x, torch.float32, "x"), _dev_ptr(out, torch.uint8, "out", tuple(x.shape)),
+                              x.numel(), _stream(stream))
+    _check(st, "ep_e4m3_encode")
+    return out
 
 
 def ep_dispatch_backward(handle: Handle, grad_recv: torch.Tensor, grad_x: Optional[torch.Tensor] = None,

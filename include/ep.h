@@ -239,6 +239,14 @@ ep_status ep_dispatch_topk(const ep_handle *handle, const float *topk_weights,
                            int32_t *recv_topk_idx, float *recv_topk_weights, int32_t *recv_slot,
                            size_t recv_rows, ep_stream_t stream);
 
+/* fp32 -> FP8 e4m3 encoding with the rounding FP8 dispatch uses (the
+ * hardware's round-to-nearest-even, saturating conversion: OCP E4M3, no
+ * infinities, values beyond +-448 and +-inf give +-448, NaN stays NaN), for
+ * callers who pre-quantise (ep_dispatch_ex accepts e4m3 input with its
+ * scales).  x: device fp32 [n]; codes: device uint8 [n]; both 16-byte
+ * aligned.  Asynchronous on `stream`. */
+ep_status ep_e4m3_encode(const float *x, uint8_t *codes, size_t n, ep_stream_t stream);
+
 /* Release a handle.  Its device memory is freed stream-ordered on the stream
  * that created it (cudaFreeAsync); work that uses the handle on other streams
  * must be ordered before that stream's current position by the caller.
