@@ -3,6 +3,9 @@
 // current device, and the stream-ordered memory pool of handles and plans.
 #pragma once
 
+#include <cstdio>
+#include <cstdlib>
+
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -26,6 +29,16 @@ inline ep_status current_device(int *dev, DeviceInfo *info) {
     if ((e = device_info(*dev, info)) != cudaSuccess) return cuda_status(e);
     if (info->cc_major != 10) return EP_ERR_NO_DEVICE;
     return EP_OK;
+}
+
+// Host logging of each call's launch shape to stderr when the environment
+// sets EP_DEBUG (to anything but "0"); read once per process.
+inline bool debug_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("EP_DEBUG");
+        return v != nullptr && v[0] != '\0' && !(v[0] == '0' && v[1] == '\0');
+    }();
+    return on;
 }
 
 // Stream-ordered pool (one per device, kept for the life of the process)

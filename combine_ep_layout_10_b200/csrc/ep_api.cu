@@ -185,6 +185,12 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     a.out_rank_tok = out_rank_tok;
     a.out_in_rank = out_in_rank;
 
+    if (debug_enabled())
+        std::fprintf(stderr,
+                     "ep: layout T=%d k=%d E=%d R=%d align=%d capacity=%d rows=%lld path=%s tiles=%d "
+                     "tile_tokens=%d threads=%d\n",
+                     T, k, E, R, A, C, (long long)n_rows, geo.small ? "one-cta" : "tiled", geo.ntiles,
+                     geo.tile_tokens, geo.small ? 1024 : geo.tile_threads);
     e = launch_layout(a, stream);  // also (re)initialises the error word
     if (e != cudaSuccess) {
         cudaFreeAsync(block, stream);
@@ -245,6 +251,10 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
     a.nchunks = nchunks;
     if ((int64_t)h->T * a.nchunks >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.nunits = h->T * a.nchunks;
+    if (debug_enabled())
+        std::fprintf(stderr, "ep: dispatch T=%d H=%d mode=%s chunk=%d units=%d num_sms=%d\n", h->T, H,
+                     a.mode == kDispatchQuantFp8 ? "bf16->e4m3" : a.mode == kDispatchCopyFp8 ? "e4m3" : "bf16",
+                     a.chunk, a.nunits, num_sms);
     cudaError_t e = launch_dispatch(a, stream);
     if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)
         e = cudaMemcpyAsync(recv_src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
@@ -282,6 +292,9 @@ ep_status ep_combine_ex(const ep_handle *h, const void *y, const float *topk_w, 
     a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
     if ((int64_t)h->T * a.blocks_per_token >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.num_sms = num_sms;
+    if (debug_enabled())
+        std::fprintf(stderr, "ep: combine T=%d H=%d blocks=%lld num_sms=%d\n", h->T, H,
+                     (long long)h->T * a.blocks_per_token, num_sms);
     return cuda_status(launch_combine(a, stream));
 }
 

@@ -87,6 +87,9 @@ ep_status ep_plan_create(const ep_handle *h, const int32_t *topk_idx, const int3
         a.recv_rows = p->recv_rows;
         a.dst = p->dst; a.pre = p->pre; a.offs = p->offs; a.recv_seg = p->recv_seg; a.recv_cnt = p->recv_cnt;
         a.err = p->err;
+        if (debug_enabled())
+            std::fprintf(stderr, "ep: plan rank=%d world=%d T=%d k=%d E=%d align=%d capacity=%d recv_rows=%lld\n",
+                         rank, world, p->T, p->k, p->E, A, C, (long long)recv_rows);
         e = launch_plan(a, stream);
     }
     if (e != cudaSuccess) {
