@@ -153,6 +153,7 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     h->experts_per_rank = E / R;
     h->tile_tokens = geo.tile_tokens;
     h->ntiles = ntiles;
+    h->layout_kernels = (ntiles == 0 || geo.small) ? 1 : 2;  // launch_layout's two paths
     h->n_rows = (int64_t)n_rows;
     h->device = dev;
     h->stream = stream;
@@ -413,6 +414,7 @@ ep_status ep_handle_get_info(const ep_handle *h, ep_handle_info *info) {
     info->expert_alignment = h->align;
     info->capacity = h->capacity;
     info->num_recv_rows = (size_t)h->n_rows;
+    info->layout_kernels = h->layout_kernels;
     return EP_OK;
 }
 

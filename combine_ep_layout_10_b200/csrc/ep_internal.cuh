@@ -142,6 +142,7 @@ constexpr int kMaxExperts = 4096;
 struct ep_handle {
     int T, k, E, R, align, capacity, experts_per_rank;
     int tile_tokens, ntiles;
+    int layout_kernels;      // kernels the layout launched (1 or 2)
     int64_t n_rows;          // receive rows the layout may use (ep_max_recv_rows)
     int device;
     cudaStream_t stream;     // the stream the handle was created (and is freed) on

@@ -65,7 +65,7 @@ class _HandleInfo(ctypes.Structure):
     _fields_ = [("num_tokens", ctypes.c_int), ("num_topk", ctypes.c_int),
                 ("num_experts", ctypes.c_int), ("num_ranks", ctypes.c_int),
                 ("expert_alignment", ctypes.c_int), ("capacity", ctypes.c_int),
-                ("num_recv_rows", ctypes.c_size_t)]
+                ("num_recv_rows", ctypes.c_size_t), ("layout_kernels", ctypes.c_int)]
 
 
 _LIB = None
@@ -202,6 +202,7 @@ class Handle:
         self.expert_alignment = info.expert_alignment
         self.capacity = info.capacity
         self.num_recv_rows = int(info.num_recv_rows)
+        self.layout_kernels = int(info.layout_kernels)
 
     @property
     def ptr(self) -> ctypes.c_void_p:

@@ -257,6 +257,7 @@ void ep_handle_free(ep_handle *handle);
 typedef struct ep_handle_info {
     int num_tokens, num_topk, num_experts, num_ranks, expert_alignment, capacity;
     size_t num_recv_rows; /* = ep_max_recv_rows(...) of this layout */
+    int layout_kernels;   /* kernels the layout launched: 1 (one CTA, or T = 0) or 2 (tiled) */
 } ep_handle_info;
 ep_status ep_handle_get_info(const ep_handle *handle, ep_handle_info *info);
 

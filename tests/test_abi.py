@@ -121,3 +121,25 @@ def test_multi_gpu_argument_errors_on_host(L):
     assert L.ep_ipc_release(None, 0) == INV
     assert L.ep_plan_check(None, None) == INV
     assert L.ep_dispatch_topk(None, None, None, None, None, 0, None) == INV
+
+
+def test_handle_info_struct_matches_the_header(tmp_path):
+    """The ctypes mirror of ep_handle_info has the C struct's size and field
+    offsets (compiled from include/ep.h with the host C compiler)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = [f for f, _ in ep._HandleInfo._fields_]
+    src = tmp_path / "info.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"ep.h\"\nint main(void) {\n"
+                   "  printf(\"%zu\\n\", sizeof(ep_handle_info));\n"
+                   + "".join("  printf(\"%%zu\\n\", offsetof(ep_handle_info, %s));\n" % f for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "info"
+    inc = os.path.join(ROOT, "include")
+    subprocess.run([cc, "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(ep._HandleInfo)] + [getattr(ep._HandleInfo, f).offset for f in fields]
+    assert got == want

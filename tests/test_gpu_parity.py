@@ -110,6 +110,16 @@ def test_layout_edge_cases(case):
     assert st == 0
     assert_layout_equal(res, md, L)
     assert res.handle.check() == ep.EP_OK
+    assert res.handle.layout_kernels == (1 if _one_cta_layout(T, k, E, R, C) else 2)
+
+
+def _one_cta_layout(T, k, E, R, C):
+    """The stated rule for the one-CTA layout: at most 1536 slots packed or
+    8192 padded, at most 512 experts, and its shared-memory plan within
+    40000 words (ids, counts, offsets, per-warp histograms, in-rank masks)."""
+    a4 = lambda n: (n + 3) // 4 * 4  # noqa: E731
+    words = a4(T * k) + a4(E) + a4(E + 1) + a4(R) + 32 * (E + 1) + T * ((R + 31) // 32)
+    return 0 < T * k <= (8192 if C else 1536) and E <= 512 and words <= 40000
 
 
 def test_layout_empty():
@@ -118,6 +128,7 @@ def test_layout_empty():
         res, md = run_layout(idx, 16, 4, 1, C)
         _, L = oracle.layout(idx.numpy(), 16, 4, 1, C)
         assert_layout_equal(res, md, L)
+        assert res.handle.layout_kernels == 1
 
 
 def test_layout_bad_expert_id_reported():
