@@ -18,7 +18,9 @@ using namespace ep;
 extern "C" {
 
 size_t ep_peer_max_recv_rows(int64_t total_tokens, int k, int E, int world, int A, int C) {
-    if (total_tokens < 0 || k < 1 || E < 1 || world < 1 || E % world != 0 || A < 1 || C < 0) return 0;
+    if (total_tokens < 0 || k < 1 || k > kMaxTopk || E < 1 || E > kMaxExperts || world < 1 || E % world != 0 ||
+        A < 1 || C < 0)
+        return 0;
     const int64_t epr = E / world;
     if (C > 0) return (size_t)(epr * C);
     return (size_t)(total_tokens * k + epr * (A - 1));

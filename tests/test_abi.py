@@ -92,6 +92,8 @@ def test_peer_max_recv_rows(L):
     assert ep.ep_peer_max_recv_rows(1000, 8, 256, 8, 1, 128) == 32 * 128
     assert ep.ep_peer_max_recv_rows(1000, 8, 255, 8) == 0      # E % world
     assert ep.ep_peer_max_recv_rows(-1, 8, 256, 8) == 0
+    assert ep.ep_peer_max_recv_rows(1000, 33, 256, 8) == 0     # k above the limit
+    assert ep.ep_peer_max_recv_rows(1000, 8, 8192, 8) == 0     # E above the limit
 
 
 def test_multi_gpu_argument_errors_on_host(L):
