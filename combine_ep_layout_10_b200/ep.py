@@ -174,11 +174,24 @@ def _dev_ptr(t: Optional[torch.Tensor], dtype, name: str, shape=None):
         raise ValueError("%s must be a CUDA tensor" % name)
     if dtype is not None and t.dtype != dtype:
         raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError("%s is on %s, but the current device is cuda:%d" % (name, t.device,
+                                                                          torch.cuda.current_device()))
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_rows(t: Optional[torch.Tensor], name: str, min_rows: int, cols: Optional[int] = None):
+    """A [rows, cols] buffer that the call indexes by receive row must hold
+    at least min_rows rows (the library cannot see a buffer's size)."""
+    if t is None:
+        return
+    if t.dim() != (1 if cols is None else 2) or t.shape[0] < min_rows or (cols is not None and t.shape[1] != cols):
+        want = "[>= %d]" % min_rows if cols is None else "[>= %d, %d]" % (min_rows, cols)
+        raise ValueError("%s must be %s, got %s" % (name, want, tuple(t.shape)))
 
 
 def ep_max_recv_rows(num_tokens: int, num_topk: int, num_experts: int,
@@ -292,6 +305,9 @@ def ep_dispatch(handle: Handle, x: torch.Tensor, use_fp8: bool, recv_x: Optional
         recv_scales = torch.empty(rows, H // 128, dtype=torch.float32, device=x.device)
     if recv_x.dim() != 2 or recv_x.shape[1] != H:
         raise ValueError("recv_x must be [rows, %d]" % H)
+    if use_fp8:
+        _check_rows(recv_scales, "recv_scales", recv_x.shape[0], H // 128)
+    _check_rows(recv_src_idx, "recv_src_idx", rows)
     st = lib().ep_dispatch(handle.ptr, _dev_ptr(x, torch.bfloat16, "x"), H, 1 if use_fp8 else 0,
                            _dev_ptr(recv_x, dt, "recv_x"),
                            _dev_ptr(recv_scales, torch.float32, "recv_scales") if use_fp8 else None,
@@ -326,6 +342,8 @@ def ep_dispatch_ex(handle: Handle, x: torch.Tensor, out_fp8: bool, x_scales: Opt
     if T != handle.num_tokens:
         raise ValueError("x has %d tokens, the handle %d" % (T, handle.num_tokens))
     in_fp8 = x.dtype == torch.float8_e4m3fn
+    if not in_fp8 and x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16 or float8_e4m3fn, got %s" % x.dtype)
     if in_fp8 and not out_fp8:
         raise ValueError("e4m3 input needs e4m3 output")
     rows = handle.num_recv_rows if recv_x is None else recv_x.shape[0]
@@ -336,15 +354,24 @@ def ep_dispatch_ex(handle: Handle, x: torch.Tensor, out_fp8: bool, x_scales: Opt
     s_row, s_grp = G, 1
     if out_fp8:
         if scale_layout == "col":
-            ld = scale_ld if scale_ld is not None else (rows + 3) // 4 * 4
-            s_row, s_grp = 1, ld
             if recv_scales is None:
+                ld = scale_ld if scale_ld is not None else (rows + 3) // 4 * 4
                 recv_scales = torch.empty(G, ld, dtype=torch.float32, device=x.device)
+            # scales of row p, group g at g * ld + p: [G, ld] with ld >= rows
+            if recv_scales.dim() != 2 or recv_scales.shape[0] != G or recv_scales.shape[1] < rows or \
+                    (scale_ld is not None and scale_ld != recv_scales.shape[1]):
+                raise ValueError("recv_scales must be [%d, scale_ld >= %d] (column-major), got %s"
+                                 % (G, rows, tuple(recv_scales.shape)))
+            s_row, s_grp = 1, recv_scales.shape[1]
         elif scale_layout == "row":
             if recv_scales is None:
                 recv_scales = torch.empty(rows, G, dtype=torch.float32, device=x.device)
+            _check_rows(recv_scales, "recv_scales", rows, G)
         else:
             raise ValueError("scale_layout must be 'row' or 'col'")
+    if recv_x.dim() != 2 or recv_x.shape[1] != H:
+        raise ValueError("recv_x must be [rows, %d]" % H)
+    _check_rows(recv_src_idx, "recv_src_idx", handle.num_recv_rows)
     st = lib().ep_dispatch_ex(handle.ptr, _dev_ptr(x, None, "x"),
                               _dev_ptr(x_scales, torch.float32, "x_scales", (T, G)) if in_fp8 else None,
                               H, EP_FORMAT_E4M3 if in_fp8 else EP_FORMAT_BF16,
@@ -421,6 +448,10 @@ def ep_combine_backward(handle: Handle, grad_out: torch.Tensor, topk_weights: to
     """Returns (grad_y [rows, H] bf16, grad_weights [T, k] fp32 or None)."""
     T, H = grad_out.shape
     rows = handle.num_recv_rows if y is None else y.shape[0]
+    if want_grad_weights and y is None:
+        raise ValueError("grad_weights need y (the expert outputs)")
+    _check_rows(y, "y", handle.num_recv_rows, H)
+    _check_rows(grad_y, "grad_y", handle.num_recv_rows, H)
     if grad_y is None:
         grad_y = torch.empty(rows, H, dtype=torch.bfloat16, device=grad_out.device)
     if want_grad_weights and grad_weights is None:
@@ -594,6 +625,8 @@ def ep_dispatch_peer(plan: Plan, peers: Peers, x: torch.Tensor, use_fp8: bool,
     (scale_ld >= the peer table's recv_rows, default recv_rows)."""
     T, H = x.shape
     in_fp8 = x.dtype == torch.float8_e4m3fn
+    if not in_fp8 and x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16 or float8_e4m3fn, got %s" % x.dtype)
     if in_fp8 and not use_fp8:
         raise ValueError("FP8 input needs FP8 output")
     if scale_layout == "row":
@@ -603,7 +636,7 @@ def ep_dispatch_peer(plan: Plan, peers: Peers, x: torch.Tensor, use_fp8: bool,
     else:
         raise ValueError("scale_layout must be 'row' or 'col'")
     st = lib().ep_dispatch_peer(plan.ptr, peers.ptr, _dev_ptr(x, x.dtype, "x", (plan.num_tokens, H)),
-                                _dev_ptr(x_scales, torch.float32, "x_scales"), H,
+                                _dev_ptr(x_scales, torch.float32, "x_scales", (plan.num_tokens, H // 128)), H,
                                 EP_FORMAT_E4M3 if in_fp8 else EP_FORMAT_BF16,
                                 EP_FORMAT_E4M3 if use_fp8 else EP_FORMAT_BF16, s_row, s_grp, num_sms,
                                 _stream(stream))

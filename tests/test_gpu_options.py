@@ -131,3 +131,41 @@ def test_option_errors():
     st = L_.ep_dispatch_ex(h.ptr, P(x.to(DEV).data_ptr()), None, w.H, 0, 1, P(recv.data_ptr()),
                            P(sc.data_ptr()), G, 1, None, rows, -1, stream)
     assert st == ep.EP_ERR_INVALID_ARG
+
+
+def test_binding_refuses_buffers_the_call_would_overrun():
+    """The library cannot see a buffer's size; the binding checks every
+    buffer indexed by receive row before anything is launched."""
+    w, x, tw, res, L = setup("prefill", 64)
+    h = res.handle
+    rows, G = h.num_recv_rows, w.H // 128
+    xd = x.to(DEV)
+    with pytest.raises(ValueError, match="recv_scales"):
+        ep.ep_dispatch(h, xd, True, recv_scales=torch.empty(rows - 1, G, device=DEV))
+    with pytest.raises(ValueError, match="recv_src_idx"):
+        ep.ep_dispatch(h, xd, False, recv_src_idx=torch.empty(rows - 1, dtype=torch.int32, device=DEV))
+    with pytest.raises(ValueError, match="recv_scales"):
+        ep.ep_dispatch_ex(h, xd, True, scale_layout="col", recv_scales=torch.empty(G, rows - 1, device=DEV))
+    with pytest.raises(ValueError, match="recv_scales"):
+        ep.ep_dispatch_ex(h, xd, True, scale_layout="col", scale_ld=rows + 8,
+                          recv_scales=torch.empty(G, rows + 4, device=DEV))
+    with pytest.raises(ValueError, match="recv_src_idx"):
+        ep.ep_dispatch_ex(h, xd, False, recv_src_idx=torch.empty(rows - 1, dtype=torch.int32, device=DEV))
+    with pytest.raises(ValueError, match="bf16 or float8_e4m3fn"):
+        ep.ep_dispatch_ex(h, xd.float(), True)
+    go = x.to(DEV)
+    with pytest.raises(ValueError, match="y must be"):
+        ep.ep_combine_backward(h, go, tw.to(DEV), y=torch.empty(rows - 1, w.H, dtype=torch.bfloat16, device=DEV))
+    with pytest.raises(ValueError, match="grad_y must be"):
+        ep.ep_combine_backward(h, go, tw.to(DEV), want_grad_weights=False,
+                               grad_y=torch.empty(rows - 1, w.H, dtype=torch.bfloat16, device=DEV))
+    with pytest.raises(ValueError, match="need y"):
+        ep.ep_combine_backward(h, go, tw.to(DEV))
+    # a column-major buffer wider than the rows, with its width as the leading dimension, is accepted
+    sc = torch.full((G, rows + 12), -1.0, device=DEV)
+    _, got, _ = ep.ep_dispatch_ex(h, xd, True, scale_layout="col", recv_scales=sc)
+    torch.cuda.synchronize()
+    _, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+    valid = L.src_idx >= 0
+    assert (got.cpu().numpy()[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
+    assert h.check() == ep.EP_OK
