@@ -23,7 +23,8 @@ combine between the ranks, NCCL collectives between the phases) as an extra
 object of the same line.
 
 `--impl reference` times the CPU oracle (the plain single-threaded C
-implementation under oracle/) on a bounded sample of the same workload.
+implementation under oracle/) on a bounded sample of the same workload per
+step, shrunk until the whole run fits a fixed time budget.
 """
 from __future__ import annotations
 
@@ -51,6 +52,8 @@ GPU_LEAD_CYCLES = 1_000_000  # ~0.5 ms spin before each timed step
 CALL_KERNELS = 2             # dispatch and combine launch one kernel each;
                              # the layout's count comes back on its handle
 HBM_FALLBACK_GBS = 6650.0
+# The reference arm's projected run time (its per-step sample shrinks to fit).
+REFERENCE_BUDGET_S = float(os.environ.get("EP_BENCH_REFERENCE_BUDGET_S", "150"))
 
 # DRAM traffic per launch from one ncu capture, keyed by the sha256 of the
 # kernel source it was taken on (stale -> reported as null).
@@ -339,10 +342,23 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     import oracle as orc
+    # Each step is a bounded sample: the dispatch and combine of the first
+    # n_tok tokens, halved (down to 64) until the whole run's projected time
+    # fits REFERENCE_BUDGET_S; the probes count as warm-up.
     n_tok = min(1024, w.T)
     x, idx, tw, y = oracle_sample_inputs(w, args.seed, n_tok)
+    probes = 0
+    while True:
+        t0 = time.perf_counter()
+        oracle_sample_step(orc, w, x, idx, tw, n_tok, y)
+        probes += 1
+        per_step = time.perf_counter() - t0
+        if n_tok <= 64 or per_step * (args.steps + args.warmup) <= REFERENCE_BUDGET_S:
+            break
+        n_tok = max(64, n_tok // 2)
+        x, idx, tw, y = oracle_sample_inputs(w, args.seed, n_tok)
     n_rows = orc.max_recv_rows(w.T, w.k, w.E, w.align, w.capacity)
-    for _ in range(args.warmup):
+    for _ in range(max(args.warmup - probes, 0)):
         oracle_sample_step(orc, w, x, idx, tw, n_tok, y)
     t0 = time.perf_counter()
     for _ in range(args.steps):

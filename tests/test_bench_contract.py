@@ -43,3 +43,12 @@ def test_reference_arm_other_ranks_exit_quietly():
                     {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"})
     assert res.returncode == 0, res.stderr
     assert res.stdout.strip() == ""
+
+
+def test_reference_arm_sample_shrinks_to_its_time_budget():
+    res = run_bench(["--impl", "reference", "--steps", "20", "--warmup", "1"],
+                    {"EP_BENCH_REFERENCE_BUDGET_S": "0.5"})
+    assert res.returncode == 0, res.stderr
+    d = json.loads(res.stdout.strip())
+    assert "first 64 tokens" in d["cpu_baseline"]["sample"]
+    assert d["steps"] == 20 and d["value"] > 0
