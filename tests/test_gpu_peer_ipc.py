@@ -41,7 +41,6 @@ def _worker(rank, world, port, q, backend="gloo", scale_layout="row"):
     result = {"rank": rank, "error": None}
     try:
         torch.cuda.set_device(0)
-        import oracle
         from oracle import multirank as MR
         from combine_ep_layout_10_b200 import ep, group
         from combine_ep_layout_10_b200 import workloads as W

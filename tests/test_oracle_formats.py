@@ -8,7 +8,6 @@ rounding are checked against
   * exact rational rounding written in tests/exact.py.
 """
 import numpy as np
-import pytest
 import torch
 
 from exact import f32, to_bf16

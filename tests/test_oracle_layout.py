@@ -9,7 +9,6 @@ checked here against formulations that share nothing with that loop:
     exactly (expert, token, slot),
   * invariants on the full-size workloads.
 """
-import itertools
 import json
 import os
 

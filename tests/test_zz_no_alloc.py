@@ -8,7 +8,6 @@ results must equal those of ep_layout (+ ep_handle_export) bit for bit, also
 on the second of two calls in a row, when the shared scratch still holds the
 first call's contents.  This file is collected last on purpose.
 """
-import numpy as np
 import pytest
 import torch
 
