@@ -76,6 +76,7 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-backward", action="store_true")
     p.add_argument("--no-overlap", action="store_true")
+    p.add_argument("--no-gemm-layout", action="store_true")
     p.add_argument("--no-ranks", action="store_true")
     p.add_argument("--ep", action="store_true",
                    help="also run expert parallelism across the job's GPUs (peer stores/loads)")
@@ -562,6 +563,10 @@ def run_ours(args, w):
     if not args.no_backward:
         backward = run_backward(w, dev, ep, idx, tw, y, flush_l2)
 
+    gemm_layout = None
+    if not args.no_gemm_layout:
+        gemm_layout = run_gemm_layout(w, dev, ep, idx, x, flush_l2)
+
     overlap = None
     if not args.no_overlap:
         overlap = run_overlap(w, dev, ep, idx, x, tw, y, flush_l2)
@@ -586,7 +591,8 @@ def run_ours(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "decode": decode, "backward": backward, "overlap": overlap, "ranks_emulated": ranks,
+            "decode": decode, "backward": backward, "gemm_layout": gemm_layout, "overlap": overlap,
+            "ranks_emulated": ranks,
             "ep_across_gpus": ep_gpus,
             "gpu_launches": launches, "clocks": clocks, "wall_s": wall,
             "host_us_per_step": host_s * 1e6,
@@ -726,6 +732,61 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
     return {"dispatch_backward": {"us": d_us, "bytes": d_bytes, "gbs": d_bytes / d_us / 1e3},
             "combine_backward": {"us": c_us, "bytes": c_bytes, "gbs": c_bytes / c_us / 1e3},
             "dispatch_topk": {"us": t_us, "bytes": t_bytes, "note": "latency-bound (~1.6 MB)"}}
+
+
+def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> dict | None:
+    """The FP8 dispatch options that serve grouped expert GEMMs
+    (ep_dispatch_ex), on the step's layout, each timed with the L2 flushed
+    before every call: scales row-major [rows, H/128] (the step's form),
+    column-major [H/128, ld] (ld = rows rounded up to 4), and pre-quantised
+    input (e4m3 codes + row-major scales, copied unchanged)."""
+    if not w.fp8:
+        return None
+    T, H, k = w.T, w.H, w.k
+    G = H // 128
+    res = ep.ep_layout(idx_dev, w.E, w.R, w.align, w.capacity)
+    h = res.handle
+    rows = h.num_recv_rows
+    ld = (rows + 3) // 4 * 4
+    recv = torch.empty(rows, H, dtype=torch.float8_e4m3fn, device=dev)
+    sc_row = torch.empty(rows, G, dtype=torch.float32, device=dev)
+    sc_col = torch.empty(G, ld, dtype=torch.float32, device=dev)
+    # pre-quantised input (plumbing, outside the timed calls): per-group scales and codes
+    xf = x_dev.float().view(T, G, 128)
+    amax = xf.abs().amax(-1).clamp_min(1e-30)
+    xs = (amax / 448.0).contiguous()
+    xq = (xf * (448.0 / amax)[..., None]).view(T, H).to(torch.float8_e4m3fn).contiguous()
+    del xf
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        ts = []
+        for i in range(steps + 3):
+            flush_l2()
+            torch.cuda._sleep(GPU_LEAD_CYCLES // 2)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if i >= 3:
+                ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ts) * 1e3
+
+    row_us = timed(lambda: ep.ep_dispatch_ex(h, x_dev, True, recv_x=recv, recv_scales=sc_row))
+    col_us = timed(lambda: ep.ep_dispatch_ex(h, x_dev, True, recv_x=recv, recv_scales=sc_col, scale_layout="col"))
+    pq_us = timed(lambda: ep.ep_dispatch_ex(h, xq, True, x_scales=xs, recv_x=recv, recv_scales=sc_row))
+    status = h.check()
+    h.free()
+    if status != ep.EP_OK:
+        raise SystemExit("gemm layout: device error %s" % ep.status_str(status))
+    V = int((idx_dev >= 0).sum().item())
+    q_bytes = T * H * 2 + T * k * 4 + V * H + V * G * 4
+    pq_bytes = T * H + T * G * 4 + T * k * 4 + V * H + V * G * 4
+    return {"scales_row_major": {"us": row_us, "bytes": q_bytes, "gbs": q_bytes / row_us / 1e3},
+            "scales_column_major": {"us": col_us, "bytes": q_bytes, "gbs": q_bytes / col_us / 1e3, "ld": ld},
+            "prequantised_input": {"us": pq_us, "bytes": pq_bytes, "gbs": pq_bytes / pq_us / 1e3}}
 
 
 def run_ranks_emulated(w, dev, ep, flush_l2, worlds=(1, 8), steps: int = 10) -> dict:
