@@ -133,6 +133,46 @@ def test_option_errors():
     assert st == ep.EP_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("prequant,num_sms,padded", [(False, 0, False), (True, 0, False), (False, 16, False),
+                                                      (False, 0, True)])
+def test_column_major_scales_large_batch(prequant, num_sms, padded):
+    """Column-major scales on a batch of over 2^20 scale stores, fused or
+    pre-quantised, with an SM budget and in padded mode: bit-exact against
+    the oracle, with tokens whose first slots are unused, a token with no
+    slot, padding rows and the leading dimension's slack untouched."""
+    w = W.WORKLOADS["prefill"].scaled(T=2400)
+    x, idx, _ = W.make_routing(w)
+    idx = idx.clone()
+    idx[::3, 0] = -1
+    idx[5, :] = -1
+    idx[7, :2] = -1
+    C = 128 if padded else 0
+    G = w.H // 128
+    assert idx.shape[0] * w.k * G >= 1 << 20
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R, 1, C)
+    st, L = oracle.layout(idx.numpy(), w.E, w.R, 1, C)
+    assert st == 0
+    rows = res.handle.num_recv_rows
+    ld = (rows + 3) // 4 * 4 + 4
+    if prequant:
+        xq, xs = oracle.quantize_rows(x)
+        xin = torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn)
+        xsd = torch.from_numpy(xs).to(DEV)
+    else:
+        xin, xsd = x.to(DEV), None
+    sc = torch.full((G, ld), -3.0, dtype=torch.float32, device=DEV)
+    recv, sc, _ = ep.ep_dispatch_ex(res.handle, xin, True, x_scales=xsd, recv_scales=sc, scale_layout="col",
+                                    num_sms=num_sms)
+    torch.cuda.synchronize()
+    q, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+    valid = L.src_idx >= 0
+    got = sc.cpu().numpy()
+    assert (got[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
+    assert (got[:, :rows].T[~valid] == -3.0).all() and (got[:, rows:] == -3.0).all()
+    assert (u8(recv)[valid] == q[valid]).all()
+    assert res.handle.check() == ep.EP_OK
+
+
 def test_binding_refuses_buffers_the_call_would_overrun():
     """The library cannot see a buffer's size; the binding checks every
     buffer indexed by receive row before anything is launched."""
