@@ -45,12 +45,15 @@
  *     legacy default stream) and is asynchronous, unless a call says it
  *     synchronises.
  *   - Argument errors are detected on the host and returned at once with
- *     nothing enqueued.  Data errors found on the device (an id outside
- *     [-1, E), a padded expert over capacity) set the
- *     handle's device error word instead; the outputs of that call are then
- *     unspecified but every device write stays inside the buffers described
- *     here.  ep_handle_check() reports the word.  No call traps, aborts or
- *     throws across the ABI.
+ *     nothing enqueued.  Data errors found on the device set the handle's
+ *     device error word instead, and the layout still completes: an id
+ *     outside [-1, E) is taken as an unused slot, and in padded mode an
+ *     expert named by more than `capacity` slots keeps its first `capacity`
+ *     slots in (token, slot) order while the rest get no row (pos -1).
+ *     Counts and is_token_in_rank count every slot that names an expert.
+ *     ep_handle_check() reports the word (a bad id before an overflow).
+ *     Every device write stays inside the buffers described here.  No call
+ *     traps, aborts or throws across the ABI.
  *   - Limits: 1 <= k <= 32, 1 <= E <= 4096, 1 <= R <= E, E % R == 0,
  *     T * k < 2^31, H % 8 == 0 (bf16) and H % 128 == 0 (FP8).
  */

@@ -168,6 +168,9 @@ void oracle_f32_to_bf16_n(const float *v, uint16_t *out, int64_t n) {
 
 static int64_t align_up64(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
+/* An expert id as the layout uses it: ids outside [-1, E) count as -1. */
+static int valid_id(int32_t e, int E) { return (e < -1 || e >= E) ? -1 : e; }
+
 /* Upper bound on the receive rows a layout can use.
  *   capacity > 0 (padded, the decoding layout): every expert owns exactly
  *     `capacity` rows, so E * capacity.
@@ -198,6 +201,14 @@ int64_t oracle_max_recv_rows(int T, int k, int E, int align, int capacity) {
  * The handle of the pages (news.hada.io, "Patrones de uso ..."; docsearch
  * item 10) carries exactly this metadata to the combine; cnt is its
  * per-expert token count list for the expert GEMMs.
+ * Two data errors still give a complete layout, and are reported in the
+ * return value:
+ *   an id outside [-1, E) is taken as an unused slot (OR_ERR_BAD_EXPERT_ID);
+ *   in padded mode, an expert named by more than `capacity` slots keeps its
+ *   first `capacity` slots in (token, slot) order and the rest get no row
+ *   (pos -1) -- the bound that num_max_tokens_per_rank (docsearch item 10)
+ *   puts on a padded buffer (OR_ERR_CAPACITY).
+ * A bad id is reported before an overflow when both occur.
  */
 int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align,
                   int capacity, int32_t *cnt, int32_t *rank_tok, uint8_t *in_rank,
@@ -215,10 +226,12 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align
     }
     int experts_per_rank = E / R;
 
-    /* Step 2: every id must name an expert or be -1. */
+    /* Step 2: every id must name an expert or be -1; any other id is
+     * reported and from here on treated as -1 (see valid_id). */
+    int bad_id = 0;
     for (int64_t s = 0; s < (int64_t)T * k; ++s) {
         if (topk_idx[s] < -1 || topk_idx[s] >= E) {
-            return OR_ERR_BAD_EXPERT_ID;
+            bad_id = 1;
         }
     }
 
@@ -229,7 +242,7 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align
     memset(in_rank, 0, (size_t)T * (size_t)R);
     for (int t = 0; t < T; ++t) {
         for (int j = 0; j < k; ++j) {
-            int e = topk_idx[(int64_t)t * k + j];
+            int e = valid_id(topk_idx[(int64_t)t * k + j], E);
             if (e < 0) {
                 continue;
             }
@@ -246,13 +259,13 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align
     }
 
     /* Step 4: expert segments and rank slices. */
-    int status = OR_OK;
+    int over = 0;
     seg[0] = 0;
     for (int e = 0; e < E; ++e) {
         if (capacity > 0) {
             seg[e + 1] = (int32_t)((int64_t)(e + 1) * capacity);
             if (cnt[e] > capacity) {
-                status = OR_ERR_CAPACITY;
+                over = 1;
             }
         } else {
             seg[e + 1] = (int32_t)(seg[e] + align_up64(cnt[e], align));
@@ -261,13 +274,12 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align
     for (int r = 0; r <= R; ++r) {
         rank_off[r] = seg[r * experts_per_rank];
     }
-    if (status != OR_OK) {
-        return status;
-    }
 
     /* Step 5: positions.  Walking tokens in ascending order and, inside a
      * token, slots in ascending order, and handing each expert its next free
-     * row, is the definition of (expert, source token, slot) order. */
+     * row, is the definition of (expert, source token, slot) order.  A padded
+     * expert whose `capacity` rows are all handed out gives no row to its
+     * later slots. */
     for (int64_t p = 0; p < n_rows; ++p) {
         src_idx[p] = -1;
     }
@@ -278,8 +290,8 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align
     for (int t = 0; t < T; ++t) {
         for (int j = 0; j < k; ++j) {
             int64_t s = (int64_t)t * k + j;
-            int e = topk_idx[s];
-            if (e < 0) {
+            int e = valid_id(topk_idx[s], E);
+            if (e < 0 || (capacity > 0 && fill[e] == capacity)) {
                 pos[s] = -1;
                 continue;
             }
@@ -290,7 +302,10 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R, int align
         }
     }
     free(fill);
-    return OR_OK;
+    if (bad_id) {
+        return OR_ERR_BAD_EXPERT_ID;
+    }
+    return over ? OR_ERR_CAPACITY : OR_OK;
 }
 
 /* ------------------------------------------------------------------------- */

@@ -138,6 +138,30 @@ def test_layout_bad_expert_id_reported():
     # the valid slots still get a consistent layout; the bad ones none
     pos = res.handle.export()["pos"].cpu().numpy()
     assert pos[1, 1] == -1 and pos[2, 0] == -1
+    # ... and the whole layout is the oracle's, which takes a bad id as an unused slot
+    st, L = oracle.layout(idx.numpy(), 4, 2, check=False)
+    assert st == 2
+    assert_layout_equal(res, res.handle.export(), L)
+
+
+@pytest.mark.parametrize("T,k,C,bad", [(10, 1, 4, False), (700, 8, 16, True), (9000, 1, 4, False),
+                                       (5000, 2, 64, True)])
+def test_layout_data_errors_match_the_oracle(T, k, C, bad):
+    """Padded overflow (an expert keeps its first `capacity` slots in (token,
+    slot) order) and invalid ids (unused slots), on the one-CTA and the tiled
+    path: the complete layout equals the oracle's and the status is the same."""
+    E, R = 16, 4
+    g = torch.Generator().manual_seed(T + k)
+    idx = torch.randint(-1, E, (T, k), generator=g, dtype=torch.int32)
+    idx[: T // 2, 0] = 3                      # expert 3 overflows
+    if bad:
+        idx[T // 3, k - 1] = E + 5
+        idx[T - 1, 0] = -7
+    res, md = run_layout(idx, E, R, 1, C)
+    st, L = oracle.layout(idx.numpy(), E, R, 1, C, check=False)
+    assert st == (2 if bad else 3)
+    assert res.handle.check() == (ep.EP_ERR_BAD_EXPERT_ID if bad else ep.EP_ERR_CAPACITY)
+    assert_layout_equal(res, md, L)
 
 
 def test_layout_errors_on_tiled_path():

@@ -28,8 +28,6 @@ def test_golden_layout(orc):
         st, L = orc.layout(idx, d["E"], d["R"], align=case["align"], capacity=case["capacity"],
                            check=False)
         assert st == case["status"], case
-        if st != 0:
-            continue
         assert L.num_tokens_per_expert.tolist() == case["num_tokens_per_expert"]
         assert L.num_tokens_per_rank.tolist() == case["num_tokens_per_rank"]
         assert L.is_token_in_rank.tolist() == case["is_token_in_rank"]
@@ -40,9 +38,12 @@ def test_golden_layout(orc):
 
 
 def brute_layout(idx, E, R, align, capacity):
-    """Independent definition by counting (no running fill counter)."""
+    """Independent definition by counting (no running fill counter).  An id
+    outside [-1, E) is an unused slot; a padded expert keeps its first
+    `capacity` slots in (token, slot) order."""
     T, k = len(idx), len(idx[0]) if len(idx) else 0
     epr = E // R
+    idx = [[e if 0 <= e < E else -1 for e in row] for row in idx]
     slots = [(t, j) for t in range(T) for j in range(k)]
     cnt = [sum(1 for (t, j) in slots if idx[t][j] == e) for e in range(E)]
     if capacity:
@@ -55,6 +56,8 @@ def brute_layout(idx, E, R, align, capacity):
         if e < 0:
             continue
         before = sum(1 for (t2, j2) in slots if (t2, j2) < (t, j) and idx[t2][j2] == e)
+        if capacity and before >= capacity:
+            continue
         pos[t][j] = seg[e] + before
     in_rank = [[int(any(idx[t][j] >= 0 and idx[t][j] // epr == r for j in range(k)))
                 for r in range(R)] for t in range(T)]
@@ -74,14 +77,17 @@ def test_bruteforce_tiny(orc, trial):
     capacity = 0
     if trial % 5 == 4:
         capacity = align * int(rng.integers(T * k // max(E, 1) + 1, T * k // max(E, 1) + 4))
+    elif trial % 10 == 3:
+        capacity = align            # tight: experts overflow and keep their first slots
     # ids in [-1, E): duplicates inside a token and unused slots on purpose
     idx = rng.integers(-1, E, size=(T, k)).astype(np.int32)
+    if trial % 7 == 6 and T:
+        idx[int(rng.integers(0, T)), int(rng.integers(0, k))] = [E, -2, E + 7][trial % 3]   # invalid id
     cnt_b, seg_b, pos_b, in_rank_b, rank_tok_b, rank_off_b = brute_layout(idx.tolist(), E, R, align, capacity)
     st, L = orc.layout(idx.reshape(T, k), E, R, align=align, capacity=capacity, check=False)
-    if capacity and max(cnt_b, default=0) > capacity:
-        assert st == 3
-        return
-    assert st == 0
+    bad = bool(((idx < -1) | (idx >= E)).any())
+    over = bool(capacity) and max(cnt_b, default=0) > capacity
+    assert st == (2 if bad else 3 if over else 0)
     assert L.num_tokens_per_expert.tolist() == cnt_b
     assert L.seg.tolist() == seg_b
     assert L.pos.reshape(T, k).tolist() == pos_b
@@ -208,6 +214,12 @@ def test_errors(orc):
     assert orc.layout(bad, 4, 2, check=False)[0] == orc.OR_ERR_BAD_EXPERT_ID
     over = np.array([[0, 1], [0, 2], [0, 3]], np.int32)
     assert orc.layout(over, 4, 2, capacity=2, check=False)[0] == orc.OR_ERR_CAPACITY
+    # both: the bad id is reported; the layout is still complete
+    both = np.array([[0, 9], [0, 2], [0, 3]], np.int32)
+    st, L = orc.layout(both, 4, 2, capacity=2, check=False)
+    assert st == orc.OR_ERR_BAD_EXPERT_ID
+    assert L.pos.tolist() == [[0, -1], [1, 4], [-1, 6]]
+    assert L.num_tokens_per_expert.tolist() == [3, 0, 1, 1]
     assert orc.max_recv_rows(10, 8, 4, 1, 0) == 80
     assert orc.max_recv_rows(10, 8, 4, 4, 0) == 92
     assert orc.max_recv_rows(10, 8, 4, 1, 16) == 64

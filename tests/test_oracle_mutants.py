@@ -24,10 +24,18 @@ SRC = os.path.join(ROOT, "oracle", "ep_oracle.c")
 # (name, text in the oracle, replacement, pins as (function, kwargs))
 MUTANTS = [
     ("positions in reversed slot order",
-     "        for (int j = 0; j < k; ++j) {\n            int64_t s = (int64_t)t * k + j;\n            int e = topk_idx[s];",
-     "        for (int j = k - 1; j >= 0; --j) {\n            int64_t s = (int64_t)t * k + j;\n            int e = topk_idx[s];",
+     "        for (int j = 0; j < k; ++j) {\n            int64_t s = (int64_t)t * k + j;\n            int e = valid_id(topk_idx[s], E);",
+     "        for (int j = k - 1; j >= 0; --j) {\n            int64_t s = (int64_t)t * k + j;\n            int e = valid_id(topk_idx[s], E);",
      # slot order only matters when a token names one expert twice
      [(PL.test_duplicates_and_unused_slots, {})] + [(PL.test_bruteforce_tiny, {"trial": t}) for t in range(20)]),
+    ("capacity overflow not reported",
+     "                over = 1;",
+     "                over = 0;",
+     [(PL.test_golden_layout, {})]),
+    ("invalid expert id not reported",
+     "            bad_id = 1;",
+     "            bad_id = 0;",
+     [(PL.test_bruteforce_tiny, {"trial": 6}), (PL.test_errors, {})]),
     ("rank of an expert taken modulo R",
      "in_rank[(int64_t)t * R + e / experts_per_rank] = 1;",
      "in_rank[(int64_t)t * R + e % R] = 1;",
