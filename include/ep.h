@@ -236,8 +236,9 @@ ep_status ep_combine_ex(const ep_handle *handle, const void *y, const float *top
  *     past num_recv_rows are not touched.
  *   recv_rows: length of those buffers, >= num_recv_rows of the handle.
  * Asynchronous, no allocation, no host synchronisation (capturable in a CUDA
- * graph with a kept handle).  If the layout found a data error the values
- * are unspecified but every write stays inside the buffers. */
+ * graph with a kept handle).  After a data error the layout is still
+ * complete (see the conventions at the top), and these values follow it:
+ * an invalid id or an over-capacity slot fills no row. */
 ep_status ep_dispatch_topk(const ep_handle *handle, const float *topk_weights,
                            int32_t *recv_topk_idx, float *recv_topk_weights, int32_t *recv_slot,
                            size_t recv_rows, ep_stream_t stream);
