@@ -202,10 +202,11 @@ inline int layout_pos_smem_words(int ntiles, int E, int R, int pos_warps, int id
 inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) {
     LayoutGeometry g;
     g.tile_tokens = EP_LAYOUT_TILE_TOKENS;
-    while ((int64_t)((T + g.tile_tokens - 1) / g.tile_tokens) * (E + R) > kLayoutMatWords &&
+    // 64-bit tile counts: T + tile_tokens - 1 overflows int for T near 2^31.
+    while (((int64_t)T + g.tile_tokens - 1) / g.tile_tokens * (E + R) > kLayoutMatWords &&
            g.tile_tokens < (1 << 29))
         g.tile_tokens *= 2;
-    g.ntiles = (T + g.tile_tokens - 1) / g.tile_tokens;
+    g.ntiles = (int)(((int64_t)T + g.tile_tokens - 1) / g.tile_tokens);
     const int rw = (R + 31) / 32;
     g.sub_tokens = 12288 / rw < g.tile_tokens ? 12288 / rw : g.tile_tokens;
     int64_t pt = ((int64_t)g.tile_tokens * k / 2 + 31) / 32 * 32;
