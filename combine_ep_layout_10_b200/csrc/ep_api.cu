@@ -206,7 +206,7 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
                          int out_format, void *recv_x, float *recv_scales, int64_t scale_row_stride,
                          int64_t scale_group_stride, int32_t *recv_src_idx, size_t recv_rows, int num_sms,
                          ep_stream_t stream) {
-    if (h == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
+    if (h == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
     const bool in_fp8 = in_format == EP_FORMAT_E4M3;
     const bool out_fp8 = out_format == EP_FORMAT_E4M3;
     if ((in_format != EP_FORMAT_BF16 && !in_fp8) || (out_format != EP_FORMAT_BF16 && !out_fp8))
@@ -270,7 +270,7 @@ ep_status ep_dispatch(const ep_handle *h, const void *x, int H, int use_fp8, voi
 
 ep_status ep_combine_ex(const ep_handle *h, const void *y, const float *topk_w, int H, size_t recv_rows,
                         void *out, int num_sms, ep_stream_t stream) {
-    if (h == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
+    if (h == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
     if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
     if (h->T > 0) {
         if (y == nullptr || out == nullptr || topk_w == nullptr) return EP_ERR_INVALID_ARG;
@@ -306,7 +306,7 @@ ep_status ep_combine(const ep_handle *h, const void *y, const float *topk_w, int
 
 ep_status ep_dispatch_backward(const ep_handle *h, const void *grad_recv, int H, size_t recv_rows,
                                void *grad_x, ep_stream_t stream) {
-    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (h == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0) return EP_ERR_INVALID_ARG;
     if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
     if (h->T > 0 && (grad_recv == nullptr || grad_x == nullptr || !aligned(grad_recv, 16) || !aligned(grad_x, 16)))
         return EP_ERR_INVALID_ARG;
@@ -331,7 +331,7 @@ ep_status ep_dispatch_backward(const ep_handle *h, const void *grad_recv, int H,
 
 ep_status ep_combine_backward(const ep_handle *h, const void *grad_out, const void *y, const float *topk_w,
                               int H, size_t recv_rows, void *grad_y, float *grad_w, ep_stream_t stream) {
-    if (h == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (h == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0) return EP_ERR_INVALID_ARG;
     if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
     if (h->T > 0) {
         if (grad_out == nullptr || topk_w == nullptr || grad_y == nullptr) return EP_ERR_INVALID_ARG;

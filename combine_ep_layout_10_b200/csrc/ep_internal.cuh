@@ -133,6 +133,7 @@ constexpr uint32_t kErrTimeout = 4u;  // reserved: no kernel waits on another to
 
 constexpr int kMaxTopk = 32;
 constexpr int kMaxExperts = 4096;
+constexpr int kMaxHidden = 1 << 24;  // channel offsets and per-row loops stay far inside int
 
 
 }  // namespace ep

@@ -290,7 +290,7 @@ ep_status ep_dispatch_topk_peer(const ep_plan *plan, const ep_peers *peers, cons
 ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const void *x, const float *x_scales,
                            int H, int in_format, int out_format, int64_t scale_row_stride,
                            int64_t scale_group_stride, int num_sms, ep_stream_t stream) {
-    if (plan == nullptr || peers == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
+    if (plan == nullptr || peers == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
     if (peers->world != plan->world || peers->recv_rows < (size_t)plan->recv_rows) return EP_ERR_INVALID_ARG;
     const bool in_fp8 = in_format == EP_FORMAT_E4M3;
     const bool out_fp8 = out_format == EP_FORMAT_E4M3;
@@ -337,7 +337,7 @@ ep_status ep_dispatch_peer(const ep_plan *plan, const ep_peers *peers, const voi
 
 ep_status ep_combine_peer(const ep_plan *plan, const ep_peers *peers, const float *topk_w, int H, void *out,
                           int num_sms, ep_stream_t stream) {
-    if (plan == nullptr || peers == nullptr || H < 8 || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
+    if (plan == nullptr || peers == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
     if (peers->world != plan->world || peers->y == nullptr || peers->recv_rows < (size_t)plan->recv_rows)
         return EP_ERR_INVALID_ARG;
     if (plan->T > 0) {
@@ -365,7 +365,7 @@ ep_status ep_combine_peer(const ep_plan *plan, const ep_peers *peers, const floa
 
 ep_status ep_combine_backward_peer(const ep_plan *plan, const ep_peers *peers, const void *grad_out,
                                    const float *topk_w, int H, float *grad_w, ep_stream_t stream) {
-    if (plan == nullptr || peers == nullptr || H < 8 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (plan == nullptr || peers == nullptr || H < 8 || H > kMaxHidden || H % 8 != 0) return EP_ERR_INVALID_ARG;
     if (peers->world != plan->world || peers->grad_y == nullptr || peers->recv_rows < (size_t)plan->recv_rows)
         return EP_ERR_INVALID_ARG;
     if (grad_w != nullptr && peers->y == nullptr) return EP_ERR_INVALID_ARG;

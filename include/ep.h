@@ -55,7 +55,7 @@
  *     Every device write stays inside the buffers described here.  No call
  *     traps, aborts or throws across the ABI.
  *   - Limits: 1 <= k <= 32, 1 <= E <= 4096, 1 <= R <= E, E % R == 0,
- *     T * k < 2^31, H % 8 == 0 (bf16) and H % 128 == 0 (FP8).
+ *     T * k < 2^31, 8 <= H <= 2^24, H % 8 == 0 (bf16) and H % 128 == 0 (FP8).
  */
 #ifndef EP_B200_EP_H
 #define EP_B200_EP_H

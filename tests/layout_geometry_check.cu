@@ -7,7 +7,8 @@
 // whole warps within 1024 threads, dynamic shared memory within the 227 KB a
 // block may opt into (static shared memory included), the per-tile count
 // matrices within the fixed scratch of the no-allocation entry point, and
-// tiles that cover the batch.  Prints one line per violation and the number
+// tiles that cover the batch; and the dispatch's work units must tile every
+// row for every hidden size up to 2^24.  Prints one line per violation and the number
 // of shapes checked; exits non-zero on any violation.
 #include <cstdint>
 #include <cstdio>
@@ -78,6 +79,24 @@ int main() {
                         if (layout_pos_smem(a) + kStaticSmem > kMaxSmem)
                             fail("position-kernel shared memory", (long long)layout_pos_smem(a));
                     }
+            }
+    // Dispatch work units: chunks of whole 8- (BF16) or 128-channel (FP8)
+    // groups, at most EP_DISPATCH_MAX_CHUNK channels (so at most 512 threads
+    // of 16 channels), that tile the row exactly.
+    for (int H = 8; H <= kMaxHidden; H = H < 65536 ? H + 8 * 37 : H * 2 + 8)
+        for (int align_ch : {8, 128})
+            for (long long T : {1LL, 7LL, 148LL, 8192LL, 1LL << 20}) {
+                if (align_ch == 128 && H % 128) continue;
+                int chunk = 0, n = 0;
+                dispatch_chunking((int)T, H, align_ch, 148, &chunk, &n);
+                ++checked;
+                const int threads = (((chunk + 15) / 16 + 31) / 32) * 32;
+                if (chunk < align_ch || chunk % align_ch || chunk > EP_DISPATCH_MAX_CHUNK || n < 1 ||
+                    (long long)n * chunk < H || (long long)(n - 1) * chunk >= H || threads > 512) {
+                    ++bad;
+                    std::printf("dispatch H=%d align=%d T=%lld: chunk %d x %d, %d threads\n", H, align_ch, T,
+                                chunk, n, threads);
+                }
             }
     std::printf("checked %lld shapes, %lld violations\n", checked, bad);
     return bad == 0 ? 0 : 1;

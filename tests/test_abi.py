@@ -67,6 +67,13 @@ def test_layout_argument_errors_on_host(L):
 def test_dispatch_combine_argument_errors_on_host(L):
     assert L.ep_dispatch(None, None, 128, 0, None, None, None, 0, None) == ep.EP_ERR_INVALID_ARG
     assert L.ep_combine(None, None, None, 128, 0, None, None) == ep.EP_ERR_INVALID_ARG
+    # hidden sizes outside [8, 2^24] or not a multiple of 8 (the handle is never dereferenced)
+    fake = ctypes.c_void_p(256)
+    for H in (0, 12, (1 << 24) + 8):
+        assert L.ep_dispatch(fake, None, H, 0, None, None, None, 0, None) == ep.EP_ERR_INVALID_ARG
+        assert L.ep_combine(fake, None, None, H, 0, None, None) == ep.EP_ERR_INVALID_ARG
+        assert L.ep_dispatch_backward(fake, None, H, 0, None, None) == ep.EP_ERR_INVALID_ARG
+        assert L.ep_combine_backward(fake, None, None, None, H, 0, None, None, None) == ep.EP_ERR_INVALID_ARG
     L.ep_handle_free(None)  # no-op
     info = ep._HandleInfo()
     assert L.ep_handle_get_info(None, ctypes.byref(info)) == ep.EP_ERR_INVALID_ARG

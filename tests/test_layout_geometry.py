@@ -6,8 +6,9 @@ shapes spanning T*k < 2^31, k <= 32, E <= 4096, every R dividing E, packed
 and padded, the geometry the library would launch must have whole-warp
 blocks within 1,024 threads, shared memory within the 227 KB a block may
 opt into, count matrices within their bound (the no-allocation scratch) and
-tiles that cover the batch exactly.  Shapes this large cannot all be run on a
-GPU; their launch shapes can all be checked here.
+tiles that cover the batch exactly; and the dispatch's work units must tile
+every row for hidden sizes up to the ABI's 2^24.  Shapes this large cannot
+all be run on a GPU; their launch shapes can all be checked here.
 """
 import os
 import subprocess
