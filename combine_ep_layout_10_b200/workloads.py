@@ -22,11 +22,13 @@ Recipe (all draws from one torch.Generator seeded with the workload seed):
      `group_size` experts by group max stay eligible; "zipf" -> logits + ln p_e;
   4. topk_idx = top-k of the scores (sorted, distinct experts), int32;
   5. topk_w = softmax over the k selected *unbiased* logits, fp32.
-Expert outputs for combine: randn(n_rows, H) rounded to bf16 from seed+1.
+Expert outputs for combine: randn(n_rows, H) rounded to bf16, drawn in seeded blocks
+(make_expert_out).
 """
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field, replace
 
 import torch
@@ -117,9 +119,30 @@ def make_x(w: Workload, seed: int) -> torch.Tensor:
 
 
 def make_expert_out(n_rows: int, H: int, seed: int) -> torch.Tensor:
-    """Synthetic expert outputs y bf16 [n_rows, H] for combine."""
-    g = torch.Generator().manual_seed(seed)
-    return torch.randn(n_rows, H, generator=g, dtype=torch.float32).to(torch.bfloat16).contiguous()
+    """Synthetic expert outputs y bf16 [n_rows, H] ~ N(0,1) for combine.
+
+    Drawn in blocks of about 2^24 values, block i from its own generator
+    seeded with seed * 1000003 + i, so the result does not depend on how many
+    host threads fill the blocks (several do, for the multi-GB full-size
+    cases)."""
+    out = torch.empty(n_rows, H, dtype=torch.bfloat16)
+    rows = max(1, (1 << 24) // max(H, 1))
+    starts = list(range(0, n_rows, rows))
+
+    def fill(i):
+        r0 = starts[i]
+        r1 = min(n_rows, r0 + rows)
+        g = torch.Generator().manual_seed(seed * 1000003 + i)
+        out[r0:r1] = torch.randn(r1 - r0, H, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+    if len(starts) <= 1:
+        for i in range(len(starts)):
+            fill(i)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1, len(starts))) as pool:
+            list(pool.map(fill, range(len(starts))))
+    return out
 
 
 def load_stats(topk_idx: torch.Tensor, E: int) -> dict:

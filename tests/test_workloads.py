@@ -43,3 +43,20 @@ def test_decode_steps_differ():
     w = W.WORKLOADS["decode"]
     a, b = W.make_x(w, 1000), W.make_x(w, 1001)
     assert a.shape == (w.T, w.H) and not torch.equal(a, b)
+
+
+def test_expert_out_blocks_are_deterministic():
+    """Expert outputs are drawn in seeded blocks: the same seed gives the same
+    tensor (whatever the thread schedule), another seed another one, and the
+    values are N(0,1) rounded to bf16."""
+    a = W.make_expert_out(9000, 4096, seed=3)   # several blocks of 4096 rows
+    b = W.make_expert_out(9000, 4096, seed=3)
+    c = W.make_expert_out(9000, 4096, seed=4)
+    assert a.dtype == torch.bfloat16 and tuple(a.shape) == (9000, 4096)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert not torch.equal(a.view(torch.int16), c.view(torch.int16))
+    # blocks differ from each other (no block reuses another's seed)
+    assert not torch.equal(a[:4096].view(torch.int16), a[4096:8192].view(torch.int16))
+    f = a.float()
+    assert abs(f.mean().item()) < 0.01 and abs(f.std().item() - 1.0) < 0.01
+    assert W.make_expert_out(0, 8, seed=1).shape == (0, 8)
