@@ -13,18 +13,24 @@
 // buffer and a fallback error word) is a file-scope __device__ array of
 // EP_NOALLOC_SCRATCH_WORDS 32-bit words: it is created when the library's
 // device code is loaded and every GPU that loads the library holds it until
-// the process exits.  Its device address is looked up once per device with
+// the process exits.  Its device address is looked up with
 // cudaGetSymbolAddress (host code cannot use the array's name as a device
-// pointer), by the first call on that device with that device current.  All
+// pointer) by the first call on a device, with that device current, and kept
+// together with the unique id of the CUDA context it belongs to.  A later call
+// that finds another context current on that device (the device was reset
+// and the library's module loaded again, possibly at another address) looks
+// the address up again, so no call launches on a stale pointer.  All
 // calls on a device share the array, so two calls whose work overlaps on the
 // GPU (different streams, no ordering between them) race on it; calls on one
 // stream are ordered and safe.  Nothing in it needs to start at zero: the
 // count kernel overwrites every tile entry the position kernel reads, and the
 // position kernel (or, for T == 0, the empty-layout kernel) overwrites the
 // error word.
+#include <cuda.h>
+
 #include <mutex>
 
-#include "ep_internal.cuh"
+#include "api_common.cuh"
 
 namespace ep {
 namespace {
@@ -34,6 +40,23 @@ static __device__ __align__(256) int32_t g_layout_scratch[EP_NOALLOC_SCRATCH_WOR
 constexpr int kMaxDevicesNoAlloc = 64;
 std::mutex g_scratch_mu;
 int32_t *g_scratch_ptr[kMaxDevicesNoAlloc];
+unsigned long long g_scratch_ctx[kMaxDevicesNoAlloc];  // context id the address belongs to
+
+// Unique id of the current CUDA context (cuCtxGetId, reached through the
+// runtime's driver entry point so that the library needs no -lcuda); false
+// when there is no current context yet or the driver lacks the call.
+bool current_context_id(unsigned long long *id) {
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetId fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<GetId>(p);
+    }();
+    return fn != nullptr && fn(nullptr, id) == CUDA_SUCCESS;
+}
 
 bool is_aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -44,15 +67,24 @@ ep_status status_of(cudaError_t e) {
     return EP_ERR_CUDA;
 }
 
-// Device address of the scratch array on `dev` (which is current).
+// Device address of the scratch array on `dev` (which is current): looked up
+// on the first call on the device and again whenever the current context is
+// not the one the kept address belongs to.
 ep_status scratch_for_device(int dev, int32_t **out) {
     if (dev < 0 || dev >= kMaxDevicesNoAlloc) return EP_ERR_INVALID_ARG;
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx);
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    if (g_scratch_ptr[dev] == nullptr || !have_ctx || g_scratch_ctx[dev] != ctx) {
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_layout_scratch);
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_layout_scratch);  // creates the context if needed
         if (e != cudaSuccess || p == nullptr) return e != cudaSuccess ? status_of(e) : EP_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<int32_t *>(p);
+        unsigned long long now = 0;
+        // Without a context id the address is not kept: every call looks it up.
+        g_scratch_ptr[dev] = current_context_id(&now) ? static_cast<int32_t *>(p) : nullptr;
+        g_scratch_ctx[dev] = now;
+        *out = static_cast<int32_t *>(p);
+        return EP_OK;
     }
     *out = g_scratch_ptr[dev];
     return EP_OK;
@@ -130,6 +162,12 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
     a.out_rank_tok = out_rank_tok;
     a.out_in_rank = out_in_rank;
 
+    if (debug_enabled())
+        std::fprintf(stderr,
+                     "ep: layout_noalloc T=%d k=%d E=%d R=%d align=%d capacity=%d rows=%lld path=%s tiles=%d "
+                     "tile_tokens=%d threads=%d scratch_words=%zu of %d\n",
+                     T, k, E, R, A, C, (long long)n_rows, geo.small ? "one-cta" : "tiled", geo.ntiles,
+                     geo.tile_tokens, geo.small ? 1024 : geo.tile_threads, need, EP_NOALLOC_SCRATCH_WORDS);
     // The layout kernels overwrite the error word; nothing else needs clearing.
     return status_of(launch_layout(a, stream));
 }
