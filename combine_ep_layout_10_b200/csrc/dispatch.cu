@@ -23,6 +23,14 @@
 //     the group's first lane copies the scale.
 // FP8 scales are written at p * s_row + g * s_grp (row-major [rows, H/128],
 // or column-major with a caller-chosen leading dimension for FP8 GEMMs).
+// Column-major scales written this way are one scattered 4-byte store per
+// (row, group): rows p and p + 1 of an expert come from different tokens and
+// so from different blocks, and nothing coalesces.  The faster form writes
+// each token's H/128 scales once to a per-token table (contiguous, small
+// enough to stay in L2) and leaves the receive rows' scales to
+// scale_fill_kernel, which walks the receive rows in order, gathers their
+// tokens' table rows into shared memory and stores every column as a
+// contiguous run.
 // Threads j < k resolve the block's k destination rows to pointers first:
 // row pos[t][j] of the local receive buffer, or, when the ranks are real GPUs
 // (PEER), row d.y of rank d.x's receive buffer, d = dst[t][j] of the plan,
@@ -56,6 +64,19 @@ __device__ __forceinline__ void st_row_v4(void *p, const uint4 &v) {
                  : "memory");
 #else
     *reinterpret_cast<uint4 *>(p) = v;
+#endif
+}
+
+// Store of a per-token table entry with an evict-last L2 policy, so that the
+// table survives the receive rows streaming through L2 until the fill pass
+// reads it.
+__device__ __forceinline__ void st_table_keep(float *p, float v) {
+#if EP_DISPATCH_TABLE_KEEP_L2
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+#else
+    *p = v;
 #endif
 }
 
@@ -104,6 +125,7 @@ template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
     __shared__ uint8_t *row_s[kMaxTopk];
     __shared__ float *srow_s[kMaxTopk];
+    __shared__ float *tok_s;  // the token's row of the per-token scale table, or nullptr
 #if EP_DISPATCH_EARLY_TRIGGER
     pdl_wait_then_trigger();
 #else
@@ -125,6 +147,7 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
             v1 = ld_nc_v4(src + 16);
         }
         slot_rows<PEER>(a, t, (size_t)a.H, row_s, srow_s);  // after the x loads are in flight
+        if (tid == 0) tok_s = a.tok_scales != nullptr ? a.tok_scales + (int64_t)t * (a.H / 128) : nullptr;
         __syncthreads();
         float f[16];
         unpack8(v0, f);
@@ -154,11 +177,12 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
                 q16.w = b[6] | (b[7] << 16);
             }
             const int g = ch / 128;
+            if (leader && tok_s != nullptr) st_table_keep(tok_s + g, scale);
             for (int j = 0; j < a.k; ++j) {
                 uint8_t *row = row_s[j];
                 if (row == nullptr) continue;
                 st_row_v4(row + ch, q16);
-                if (leader) srow_s[j][(int64_t)g * a.s_grp] = scale;
+                if (leader && srow_s[j] != nullptr) srow_s[j][(int64_t)g * a.s_grp] = scale;
             }
         }
         if (!LOOP) break;
@@ -200,7 +224,7 @@ __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) 
                 uint8_t *row = row_s[j];
                 if (row == nullptr) continue;
                 st_row_v4(row + ch, v);
-                if (leader) srow_s[j][(int64_t)g * a.s_grp] = scale;
+                if (leader && srow_s[j] != nullptr) srow_s[j][(int64_t)g * a.s_grp] = scale;
             }
         }
         if (!LOOP) break;
@@ -271,9 +295,141 @@ cudaError_t launch_dispatch_impl(const DispatchArgs &a, cudaStream_t st) {
     return launch_kernel(kernel, (unsigned)grid, threads, 0, st, a);
 }
 
+// Column-major scales from the per-token table.  A block takes tiles of
+// kFillRows consecutive receive rows and up to kFillGroups groups: it reads
+// the tiles' source tokens, gathers each token's table row (contiguous
+// floats; 16-byte loads when rows allow, all of a thread's loads issued
+// before any is used, so a tile costs about one memory round trip) into
+// shared memory and then stores every group's column of the tile as one
+// contiguous run of up to kFillRows floats.  The table is read with an
+// evict-first L2 policy: each entry is dead once its rows are filled.
+constexpr int kFillRows = 128;
+constexpr int kFillGroups = 64;
+constexpr int kFillThreads = 256;
+constexpr int kFillVecPerThread = kFillRows / (2 * (kFillThreads / 32));  // rows of a thread in the 16-byte gather
+static_assert(kFillGroups / 4 <= 16, "a half-warp holds one row's 16-byte pieces");
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ float4 ld_table_v4(const float *p, uint64_t pol) {
+    float4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p), "l"(pol));
+    return r;
+}
+
+__device__ __forceinline__ float ld_table(const float *p, uint64_t pol) {
+    float r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(r) : "l"(p), "l"(pol));
+    return r;
+}
+
+__global__ void __launch_bounds__(kFillThreads) scale_fill_kernel(ScaleFillArgs a) {
+    __shared__ float tile_s[kFillRows * (kFillGroups + 1)];
+    __shared__ int32_t src_s[kFillRows];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    constexpr int kWarps = kFillThreads / 32;
+    const int64_t ntiles = (a.n_rows + kFillRows - 1) / kFillRows;
+    // The source tokens of the first tile are read before the wait for the
+    // dispatch: the layout wrote them, and it completed before the dispatch
+    // (this kernel's predecessor) began.  The table is read only after it.
+    if (blockIdx.x < ntiles) {
+        const int64_t p0 = (int64_t)blockIdx.x * kFillRows;
+        const int n = (int)min((int64_t)kFillRows, a.n_rows - p0);
+        for (int i = tid; i < n; i += kFillThreads) src_s[i] = __ldg(a.src_idx + p0 + i);
+    }
+    pdl_wait_then_trigger();
+    const uint64_t pol = l2_evict_first_policy();
+    const int g0 = blockIdx.y * kFillGroups;
+    const int gn = min(kFillGroups, a.G - g0);
+    const int ldt = gn | 1;  // odd row stride: the column reads below hit distinct banks
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t p0 = tile * kFillRows;
+        const int n = (int)min((int64_t)kFillRows, a.n_rows - p0);
+        if (tile != blockIdx.x)
+            for (int i = tid; i < n; i += kFillThreads) src_s[i] = __ldg(a.src_idx + p0 + i);
+        __syncthreads();
+        if (a.vec_in) {
+            // 16-byte pieces (G % 4 == 0, so gn % 4 == 0 and every table row is
+            // 16-byte aligned): a warp takes two rows at a time, a half-warp per
+            // row, a lane per piece (gn / 4 <= 16); no integer division.
+            const int gv = gn >> 2;
+            const int c = lane & 15;
+            float4 v[kFillVecPerThread];
+#pragma unroll
+            for (int q = 0; q < kFillVecPerThread; ++q) {
+                const int i = (q * kWarps + warp) * 2 + (lane >> 4);
+                v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < n && c < gv) {
+                    const int32_t t = src_s[i];
+                    if (t >= 0) v[q] = ld_table_v4(a.table + (int64_t)t * a.G + g0 + 4 * c, pol);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < kFillVecPerThread; ++q) {
+                const int i = (q * kWarps + warp) * 2 + (lane >> 4);
+                if (i < n && c < gv) {
+                    float *d = tile_s + i * ldt + 4 * c;
+                    d[0] = v[q].x;
+                    d[1] = v[q].y;
+                    d[2] = v[q].z;
+                    d[3] = v[q].w;
+                }
+            }
+        } else {
+            // A warp per row, a lane per group (two passes of 32 groups).
+            for (int i = warp; i < n; i += kWarps) {
+                const int32_t t = src_s[i];
+#pragma unroll
+                for (int h = 0; h < kFillGroups; h += 32) {
+                    const int g = h + lane;
+                    if (g < gn) tile_s[i * ldt + g] = t >= 0 ? ld_table(a.table + (int64_t)t * a.G + g0 + g, pol) : 0.0f;
+                }
+            }
+        }
+        __syncthreads();
+        // Store: a warp per column of the tile, consecutive lanes on consecutive rows.
+        for (int g = warp; g < gn; g += kWarps) {
+            float *col = a.scales + (int64_t)(g0 + g) * a.ld + p0;
+#pragma unroll
+            for (int i0 = 0; i0 < kFillRows; i0 += 32) {
+                const int i = i0 + lane;
+                if (i < n && src_s[i] >= 0) col[i] = tile_s[i * ldt + g];
+            }
+        }
+        __syncthreads();  // src_s / tile_s are rewritten by the next tile
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t st) { return launch_dispatch_impl<false>(a, st); }
+
+cudaError_t launch_scale_fill(const ScaleFillArgs &a, cudaStream_t st) {
+    if (a.n_rows == 0 || a.G == 0) return cudaSuccess;
+    if (a.vec_in && (a.G % 4 != 0 || (reinterpret_cast<uintptr_t>(a.table) & 15u) != 0))
+        return cudaErrorInvalidValue;
+    const int64_t ntiles = (a.n_rows + kFillRows - 1) / kFillRows;
+    const int gchunks = (a.G + kFillGroups - 1) / kFillGroups;
+    int64_t grid = ntiles;
+    if (a.num_sms > 0) {
+        int per_sm = 0;
+        cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scale_fill_kernel, kFillThreads, 0);
+        if (err != cudaSuccess) return err;
+        const int64_t cap = (int64_t)a.num_sms * (per_sm > 0 ? per_sm : 1);
+        const int64_t per_chunk = (cap + gchunks - 1) / gchunks;  // blocks of the grid's x dimension
+        if (per_chunk < grid) grid = per_chunk;
+    }
+    if (grid > 0x7fffffff) grid = 0x7fffffff;
+    return launch_kernel(scale_fill_kernel, dim3((unsigned)grid, (unsigned)gchunks), kFillThreads, 0, st, a);
+}
 
 cudaError_t launch_dispatch_peer(const DispatchArgs &a, cudaStream_t st) { return launch_dispatch_impl<true>(a, st); }
 

@@ -153,7 +153,7 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     h->experts_per_rank = E / R;
     h->tile_tokens = geo.tile_tokens;
     h->ntiles = ntiles;
-    h->layout_kernels = (ntiles == 0 || geo.small) ? 1 : 2;  // launch_layout's two paths
+
     h->n_rows = (int64_t)n_rows;
     h->device = dev;
     h->stream = stream;
@@ -185,12 +185,15 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     a.out_cnt = out_cnt;
     a.out_rank_tok = out_rank_tok;
     a.out_in_rank = out_in_rank;
+    h->layout_path = ntiles == 0 ? kLayoutPathEmpty : geo.small ? kLayoutPathOneCta : kLayoutPathTiled;
+    h->layout_kernels = h->layout_path == kLayoutPathTiled ? 2 : 1;
 
     if (debug_enabled())
         std::fprintf(stderr,
                      "ep: layout T=%d k=%d E=%d R=%d align=%d capacity=%d rows=%lld path=%s tiles=%d "
                      "tile_tokens=%d threads=%d\n",
-                     T, k, E, R, A, C, (long long)n_rows, geo.small ? "one-cta" : "tiled", geo.ntiles,
+                     T, k, E, R, A, C, (long long)n_rows,
+                     geo.small ? "one-cta" : "tiled", geo.ntiles,
                      geo.tile_tokens, geo.small ? 1024 : geo.tile_threads);
     e = launch_layout(a, stream);  // also (re)initialises the error word
     if (e != cudaSuccess) {
@@ -215,11 +218,13 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
     if (out_fp8 && H % 128 != 0) return EP_ERR_INVALID_ARG;
     if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
     const int64_t G = H / 128;
+    bool col_fill = false;  // pre-quantised input, column-major scales: codes copied, then the fill pass
     if (out_fp8) {
         // Non-overlapping scale layouts only: row-major-like or column-major-like.
         const bool row_like = scale_group_stride == 1 && scale_row_stride >= G;
         const bool col_like = scale_row_stride == 1 && scale_group_stride >= (int64_t)recv_rows;
         if (!(row_like || col_like)) return EP_ERR_INVALID_ARG;
+        col_fill = in_fp8 && col_like && !row_like;
     }
     if (h->T > 0) {
         if (x == nullptr || recv_x == nullptr || !aligned(x, 16) || !aligned(recv_x, 16))
@@ -242,7 +247,7 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
     a.x_scales = x_scales;
     a.pos = h->pos;
     a.recv = static_cast<uint8_t *>(recv_x);
-    a.scales = recv_scales;
+    a.scales = col_fill ? nullptr : recv_scales;
     a.s_row = scale_row_stride;
     a.s_grp = scale_group_stride;
     a.mode = !out_fp8 ? kDispatchCopyBf16 : in_fp8 ? kDispatchCopyFp8 : kDispatchQuantFp8;
@@ -257,6 +262,76 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
                      a.mode == kDispatchQuantFp8 ? "bf16->e4m3" : a.mode == kDispatchCopyFp8 ? "e4m3" : "bf16",
                      a.chunk, a.nunits, num_sms);
     cudaError_t e = launch_dispatch(a, stream);
+    if (e == cudaSuccess && col_fill && h->T > 0) {
+        // The input's own scale table [T, H/128] is the fill pass's source.
+        ScaleFillArgs f{};
+        f.src_idx = h->src_idx;
+        f.table = x_scales;
+        f.scales = recv_scales;
+        f.ld = scale_group_stride;
+        f.n_rows = h->n_rows;
+        f.G = (int)G;
+        f.num_sms = num_sms;
+        f.vec_in = G % 4 == 0 && aligned(x_scales, 16);
+        e = launch_scale_fill(f, stream);
+    }
+    if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)
+        e = cudaMemcpyAsync(recv_src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
+    return cuda_status(e);
+}
+
+ep_status ep_dispatch_fp8_colmajor(const ep_handle *h, const void *x, int H, void *recv_x, float *recv_scales,
+                                   int64_t scale_ld, float *token_scales, int32_t *recv_src_idx,
+                                   size_t recv_rows, int num_sms, ep_stream_t stream) {
+    if (h == nullptr || H < 128 || H > kMaxHidden || H % 128 != 0 || num_sms < 0) return EP_ERR_INVALID_ARG;
+    if (scale_ld < 1 || recv_rows > ((size_t)1 << 62) || scale_ld < (int64_t)recv_rows) return EP_ERR_INVALID_ARG;
+    if (recv_rows < (size_t)h->n_rows) return EP_ERR_INVALID_ARG;
+    if (h->T > 0) {
+        if (x == nullptr || recv_x == nullptr || recv_scales == nullptr || token_scales == nullptr)
+            return EP_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(recv_scales, 4) || !aligned(token_scales, 4))
+            return EP_ERR_INVALID_ARG;
+    }
+    if (recv_src_idx != nullptr && !aligned(recv_src_idx, 4)) return EP_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    ep_status st = current_device(&dev, &info);
+    if (st != EP_OK) return st;
+    if (dev != h->device) return EP_ERR_INVALID_ARG;
+
+    int chunk, nchunks;
+    dispatch_chunking(h->T, H, 128, info.num_sms, &chunk, &nchunks);
+    if ((int64_t)h->T * nchunks >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
+    DispatchArgs a{};
+    a.x = static_cast<const uint8_t *>(x);
+    a.pos = h->pos;
+    a.recv = static_cast<uint8_t *>(recv_x);
+    a.scales = nullptr;         // the receive rows' scales come from the fill pass
+    a.tok_scales = token_scales;
+    a.s_row = 1;
+    a.s_grp = scale_ld;
+    a.mode = kDispatchQuantFp8;
+    a.num_sms = num_sms;
+    a.T = h->T; a.k = h->k; a.H = H;
+    a.chunk = chunk;
+    a.nchunks = nchunks;
+    a.nunits = h->T * nchunks;
+    if (debug_enabled())
+        std::fprintf(stderr, "ep: dispatch_fp8_colmajor T=%d H=%d chunk=%d units=%d ld=%lld num_sms=%d\n", h->T,
+                     H, a.chunk, a.nunits, (long long)scale_ld, num_sms);
+    cudaError_t e = launch_dispatch(a, stream);
+    if (e == cudaSuccess && h->T > 0) {
+        ScaleFillArgs f{};
+        f.src_idx = h->src_idx;
+        f.table = token_scales;
+        f.scales = recv_scales;
+        f.ld = scale_ld;
+        f.n_rows = h->n_rows;
+        f.G = H / 128;
+        f.num_sms = num_sms;
+        f.vec_in = f.G % 4 == 0 && aligned(token_scales, 16);
+        e = launch_scale_fill(f, stream);
+    }
     if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)
         e = cudaMemcpyAsync(recv_src_idx, h->src_idx, (size_t)h->n_rows * 4, cudaMemcpyDeviceToDevice, stream);
     return cuda_status(e);
@@ -415,6 +490,7 @@ ep_status ep_handle_get_info(const ep_handle *h, ep_handle_info *info) {
     info->capacity = h->capacity;
     info->num_recv_rows = (size_t)h->n_rows;
     info->layout_kernels = h->layout_kernels;
+    info->layout_path = h->layout_path;
     return EP_OK;
 }
 

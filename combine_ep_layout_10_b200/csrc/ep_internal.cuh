@@ -23,6 +23,9 @@
 #ifndef EP_DISPATCH_STORE_CS      // dispatch: evict-first (.cs) stores of the receive rows
 #define EP_DISPATCH_STORE_CS 0
 #endif
+#ifndef EP_DISPATCH_TABLE_KEEP_L2  // dispatch: per-token scale table stored with an evict-last L2 policy
+#define EP_DISPATCH_TABLE_KEEP_L2 1
+#endif
 #ifndef EP_COMBINE_THREADS        // threads per combine block
 #define EP_COMBINE_THREADS 128
 #endif
@@ -144,6 +147,7 @@ struct ep_handle {
     int T, k, E, R, align, capacity, experts_per_rank;
     int tile_tokens, ntiles;
     int layout_kernels;      // kernels the layout launched (1 or 2)
+    int layout_path;         // kLayoutPath*
     int64_t n_rows;          // receive rows the layout may use (ep_max_recv_rows)
     int device;
     cudaStream_t stream;     // the stream the handle was created (and is freed) on
@@ -235,6 +239,11 @@ struct LayoutArgs {
     uint8_t *out_in_rank;
 };
 
+// Layout paths, as ep_handle_info reports them.
+constexpr int kLayoutPathEmpty = 0;
+constexpr int kLayoutPathOneCta = 1;
+constexpr int kLayoutPathTiled = 2;  // layout_count_kernel + layout_pos_kernel
+
 constexpr int kDispatchCopyBf16 = 0;  // bf16 in, bf16 rows out
 constexpr int kDispatchQuantFp8 = 1;  // bf16 in, e4m3 rows + scales out (quantised here)
 constexpr int kDispatchCopyFp8 = 2;   // e4m3 + scales in (already quantised), copied out
@@ -256,6 +265,27 @@ struct DispatchArgs {
     const int2 *dst;                 // [T, k] (rank, row) of each slot, rank -1 if none
     uint8_t *const *peer_recv;       // [world] device pointers to every rank's receive buffer
     float *const *peer_scales;       // [world] ... scale buffers (FP8), or nullptr
+    // Per-token scale table [T, H/128] row-major, written by the quantising
+    // kernel when not null (kDispatchQuantFp8; local addressing only).  With
+    // scales == nullptr no receive row gets a scale: a fill pass
+    // (launch_scale_fill) writes them from the table afterwards.
+    float *tok_scales;
+};
+
+// Column-order fill of column-major FP8 scales from a per-token table:
+// scales[g * ld + p] = table[src_idx[p] * G + g] for every receive row p with
+// src_idx[p] >= 0 (padding rows are not written).  Launched right after a
+// dispatch kernel of the same handle: it reads src_idx before waiting for
+// that kernel (the layout that wrote src_idx completed before it).
+struct ScaleFillArgs {
+    const int32_t *src_idx;  // [n_rows] (handle)
+    const float *table;      // [T, G] row-major per-token scales
+    float *scales;           // column-major: element (p, g) at g * ld + p
+    int64_t ld;              // >= n_rows
+    int64_t n_rows;
+    int G;                   // H / 128
+    int num_sms;             // 0: one block per tile; else grid capped
+    bool vec_in;             // table rows read as 16-byte vectors (G % 4 == 0, table 16-byte aligned)
 };
 
 struct CombineArgs {
@@ -385,6 +415,7 @@ size_t layout_count_smem(const LayoutArgs &a);
 size_t layout_small_smem(const LayoutArgs &a);
 size_t layout_pos_smem(const LayoutArgs &a);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
+cudaError_t launch_scale_fill(const ScaleFillArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBwdArgs &a, cudaStream_t s);
 cudaError_t launch_recv_topk(const RecvTopkArgs &a, cudaStream_t s);

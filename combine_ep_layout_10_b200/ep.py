@@ -8,8 +8,8 @@ the calls raise.
 
 The names follow the C ABI: ep_max_recv_rows, ep_layout, ep_dispatch,
 ep_combine, ep_handle_free (plus the handle accessors), the option, backward
-and per-row calls (ep_dispatch_ex, ep_combine_ex, ep_dispatch_backward,
-ep_combine_backward, ep_dispatch_topk, ep_layout_noalloc) and the multi-GPU
+and per-row calls (ep_dispatch_ex, ep_dispatch_fp8_colmajor, ep_combine_ex,
+ep_dispatch_backward, ep_combine_backward, ep_dispatch_topk, ep_layout_noalloc) and the multi-GPU
 calls (ep_plan_create, Peers, ep_dispatch_peer, ep_combine_peer,
 ep_combine_backward_peer, ipc_export / ipc_import / ipc_release).
 """
@@ -42,7 +42,7 @@ ABI_SYMBOLS = (
     "ep_status_str", "ep_max_recv_rows", "ep_layout", "ep_dispatch", "ep_combine",
     "ep_handle_free", "ep_handle_get_info", "ep_handle_export", "ep_handle_counts_host",
     "ep_handle_check", "ep_layout_noalloc", "ep_dispatch_backward", "ep_combine_backward",
-    "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk",
+    "ep_dispatch_ex", "ep_combine_ex", "ep_dispatch_topk", "ep_dispatch_fp8_colmajor",
     "ep_peer_max_recv_rows", "ep_plan_create", "ep_plan_free", "ep_plan_export", "ep_plan_recv_rows_host",
     "ep_plan_check", "ep_peers_create", "ep_peers_free", "ep_dispatch_peer", "ep_combine_peer",
     "ep_combine_backward_peer", "ep_peers_set_topk", "ep_dispatch_topk_peer", "ep_e4m3_encode",
@@ -50,6 +50,11 @@ ABI_SYMBOLS = (
 )
 
 EP_IPC_HANDLE_BYTES = 64
+
+#: How a layout ran (ep_handle_info.layout_path).
+EP_LAYOUT_PATH_EMPTY = 0
+EP_LAYOUT_PATH_ONE_CTA = 1
+EP_LAYOUT_PATH_TILED = 2
 
 EP_FORMAT_BF16 = 0
 EP_FORMAT_E4M3 = 1
@@ -65,7 +70,8 @@ class _HandleInfo(ctypes.Structure):
     _fields_ = [("num_tokens", ctypes.c_int), ("num_topk", ctypes.c_int),
                 ("num_experts", ctypes.c_int), ("num_ranks", ctypes.c_int),
                 ("expert_alignment", ctypes.c_int), ("capacity", ctypes.c_int),
-                ("num_recv_rows", ctypes.c_size_t), ("layout_kernels", ctypes.c_int)]
+                ("num_recv_rows", ctypes.c_size_t), ("layout_kernels", ctypes.c_int),
+                ("layout_path", ctypes.c_int)]
 
 
 _LIB = None
@@ -109,6 +115,8 @@ def lib() -> ctypes.CDLL:
         I64 = ctypes.c_int64
         L.ep_dispatch_ex.argtypes = [P, P, P, I, I, I, P, P, I64, I64, P, S, I, P]
         L.ep_dispatch_ex.restype = I
+        L.ep_dispatch_fp8_colmajor.argtypes = [P, P, I, P, P, I64, P, P, S, I, P]
+        L.ep_dispatch_fp8_colmajor.restype = I
         L.ep_combine_ex.argtypes = [P, P, P, I, S, P, I, P]
         L.ep_dispatch_topk.argtypes = [P, P, P, P, P, S, P]
         L.ep_dispatch_topk.restype = I
@@ -216,6 +224,7 @@ class Handle:
         self.capacity = info.capacity
         self.num_recv_rows = int(info.num_recv_rows)
         self.layout_kernels = int(info.layout_kernels)
+        self.layout_path = int(info.layout_path)
 
     @property
     def ptr(self) -> ctypes.c_void_p:
@@ -382,6 +391,42 @@ def ep_dispatch_ex(handle: Handle, x: torch.Tensor, out_fp8: bool, x_scales: Opt
                               rows, num_sms, _stream(stream))
     _check(st, "ep_dispatch_ex")
     return recv_x, (recv_scales if out_fp8 else None), recv_src_idx
+
+
+def ep_dispatch_fp8_colmajor(handle: Handle, x: torch.Tensor, recv_x: Optional[torch.Tensor] = None,
+                             recv_scales: Optional[torch.Tensor] = None, token_scales: Optional[torch.Tensor] = None,
+                             recv_src_idx: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None):
+    """FP8 dispatch with column-major scales ([H/128, ld], ld >= rows; the
+    grouped-GEMM layout) through a per-token scale table.  Returns (recv_x,
+    recv_scales [H/128, ld], token_scales [T, H/128], recv_src_idx or None)."""
+    T, H = x.shape
+    if T != handle.num_tokens:
+        raise ValueError("x has %d tokens, the handle %d" % (T, handle.num_tokens))
+    if H % 128 != 0:
+        raise ValueError("FP8 dispatch needs H %% 128 == 0, got %d" % H)
+    G = H // 128
+    rows = handle.num_recv_rows if recv_x is None else recv_x.shape[0]
+    if recv_x is None:
+        recv_x = torch.empty(rows, H, dtype=torch.float8_e4m3fn, device=x.device)
+    if recv_x.dim() != 2 or recv_x.shape[1] != H or rows < handle.num_recv_rows:
+        raise ValueError("recv_x must be [>= %d, %d], got %s" % (handle.num_recv_rows, H, tuple(recv_x.shape)))
+    if recv_scales is None:
+        recv_scales = torch.empty(G, (rows + 3) // 4 * 4, dtype=torch.float32, device=x.device)
+    if recv_scales.dim() != 2 or recv_scales.shape[0] != G or recv_scales.shape[1] < rows:
+        raise ValueError("recv_scales must be [%d, scale_ld >= %d] (column-major), got %s"
+                         % (G, rows, tuple(recv_scales.shape)))
+    if token_scales is None:
+        token_scales = torch.empty(T, G, dtype=torch.float32, device=x.device)
+    _check_rows(recv_src_idx, "recv_src_idx", handle.num_recv_rows)
+    st = lib().ep_dispatch_fp8_colmajor(handle.ptr, _dev_ptr(x, torch.bfloat16, "x"), H,
+                                        _dev_ptr(recv_x, torch.float8_e4m3fn, "recv_x"),
+                                        _dev_ptr(recv_scales, torch.float32, "recv_scales"),
+                                        recv_scales.shape[1],
+                                        _dev_ptr(token_scales, torch.float32, "token_scales", (T, G)),
+                                        _dev_ptr(recv_src_idx, torch.int32, "recv_src_idx"),
+                                        rows, num_sms, _stream(stream))
+    _check(st, "ep_dispatch_fp8_colmajor")
+    return recv_x, recv_scales, token_scales, recv_src_idx
 
 
 def ep_combine_ex(handle: Handle, y: torch.Tensor, topk_weights: torch.Tensor,

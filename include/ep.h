@@ -92,8 +92,13 @@ const char *ep_status_str(ep_status status);
 
 /* Upper bound on the receive rows a layout with these parameters can use:
  * E * capacity in padded mode, T*k + E*(expert_alignment-1) in packed mode.
- * recv_x / y must have at least this many rows.  Host only, pure.  Returns 0
- * for invalid arguments. */
+ * recv_x / y must have at least this many rows.  This is the receive-buffer
+ * bound the pages' dispatch takes as num_max_tokens_per_rank ("DeepEP
+ * (DeepEveryParallel) Documentation", item 10: the per-rank receive capacity
+ * is an argument of dispatch, so the buffers can be sized before any routing
+ * is known); with `capacity` > 0 the bound is the padded per-expert layout of
+ * the decoding case (item 3).  Host only, pure.  Returns 0 for invalid
+ * arguments. */
 size_t ep_max_recv_rows(int num_tokens, int num_topk, int num_experts,
                         int expert_alignment, int capacity);
 
@@ -204,7 +209,11 @@ ep_status ep_combine_backward(const ep_handle *handle, const void *grad_out, con
  *     uses H/128) and column-major (row stride 1, group stride >= recv_rows,
  *     e.g. recv_rows rounded up to a multiple of 4 for 16-byte aligned
  *     columns).  The buffer must hold (recv_rows-1)*row_stride +
- *     (H/128-1)*group_stride + 1 floats.
+ *     (H/128-1)*group_stride + 1 floats.  Column-major scales of e4m3 input
+ *     are written by a second kernel from x_scales in receive-row order
+ *     (contiguous runs per column); of quantised-here input, by the
+ *     dispatch itself, one 4-byte store per row and group
+ *     (ep_dispatch_fp8_colmajor is the faster call for that case).
  *   num_sms: 0 = no limit (one block per token chunk); n > 0 = at most the
  *     blocks n SMs can hold at once, looping over the work, so that
  *     concurrent kernels on other streams keep the remaining SMs' worth of
@@ -214,6 +223,27 @@ ep_status ep_dispatch_ex(const ep_handle *handle, const void *x, const float *x_
                          int in_format, int out_format, void *recv_x, float *recv_scales,
                          int64_t scale_row_stride, int64_t scale_group_stride,
                          int32_t *recv_src_idx, size_t recv_rows, int num_sms, ep_stream_t stream);
+
+/* FP8 dispatch with column-major scales, the layout a grouped FP8 GEMM reads
+ * ([hada] "Cambios clave de la versión V2": a GEMM layout), written the fast
+ * way.  Codes, scales and rules as ep_dispatch with use_fp8 != 0; the scale
+ * of receive row p and group g goes to recv_scales[g * scale_ld + p].
+ *   scale_ld: leading dimension of recv_scales, >= recv_rows (e.g. recv_rows
+ *     rounded up to a multiple of 4 for 16-byte aligned columns); the buffer
+ *     holds (H/128 - 1) * scale_ld + recv_rows floats.
+ *   token_scales: device fp32 [T, H/128] row-major, written: the scale of every
+ *     token and group (the values the token's receive rows get).  Besides
+ *     being an output, it is the table the second kernel reads.
+ * Two kernels: the dispatch writes the codes of every receive row and each
+ * token's scales once, into token_scales; a second kernel walks the receive
+ * rows in order and stores recv_scales column by column as contiguous runs.
+ * (ep_dispatch_ex with a column-major layout gives the same values with one
+ * scattered 4-byte store per row and group, which is slower.)  Padding rows
+ * are not written.  num_sms as in ep_dispatch_ex.  No allocation, no host
+ * synchronisation. */
+ep_status ep_dispatch_fp8_colmajor(const ep_handle *handle, const void *x, int hidden, void *recv_x,
+                                   float *recv_scales, int64_t scale_ld, float *token_scales,
+                                   int32_t *recv_src_idx, size_t recv_rows, int num_sms, ep_stream_t stream);
 
 /* Combine with an SM budget: as ep_combine, with num_sms as in ep_dispatch_ex. */
 ep_status ep_combine_ex(const ep_handle *handle, const void *y, const float *topk_weights,
@@ -251,10 +281,13 @@ ep_status ep_dispatch_topk(const ep_handle *handle, const float *topk_weights,
  * aligned.  Asynchronous on `stream`. */
 ep_status ep_e4m3_encode(const float *x, uint8_t *codes, size_t n, ep_stream_t stream);
 
-/* Release a handle.  Its device memory is freed stream-ordered on the stream
- * that created it (cudaFreeAsync); work that uses the handle on other streams
- * must be ordered before that stream's current position by the caller.
- * NULL is a no-op. */
+/* Release a handle: the end of the pages' EPHandle's life ("DeepEP
+ * (DeepEveryParallel) Documentation", items 3 and 10: a handle returned by
+ * dispatch is passed to combine and, while the routing does not change, to
+ * later dispatches; here the caller says when it is no longer needed).  Its
+ * device memory is freed stream-ordered on the stream that created it
+ * (cudaFreeAsync); work that uses the handle on other streams must be ordered
+ * before that stream's current position by the caller.  NULL is a no-op. */
 void ep_handle_free(ep_handle *handle);
 
 /* Handle geometry (host only, no device work). */
@@ -262,7 +295,11 @@ typedef struct ep_handle_info {
     int num_tokens, num_topk, num_experts, num_ranks, expert_alignment, capacity;
     size_t num_recv_rows; /* = ep_max_recv_rows(...) of this layout */
     int layout_kernels;   /* kernels the layout launched: 1 (one CTA, or T = 0) or 2 (tiled) */
+    int layout_path;      /* EP_LAYOUT_PATH_*: how the layout ran */
 } ep_handle_info;
+#define EP_LAYOUT_PATH_EMPTY 0   /* T == 0 */
+#define EP_LAYOUT_PATH_ONE_CTA 1 /* small problems: the whole layout in one CTA */
+#define EP_LAYOUT_PATH_TILED 2   /* one CTA per tile of tokens, two kernels */
 ep_status ep_handle_get_info(const ep_handle *handle, ep_handle_info *info);
 
 /* Copy the handle's metadata into caller buffers (device-to-device, async on
@@ -278,13 +315,19 @@ ep_status ep_handle_counts_host(const ep_handle *handle, int32_t *host_counts,
                                 ep_stream_t stream);
 
 /* Read the handle's device error word after the work enqueued on `stream`
- * so far.  Synchronises `stream`.  Returns EP_OK, EP_ERR_BAD_EXPERT_ID,
- * EP_ERR_CAPACITY or EP_ERR_TIMEOUT (the first set, in that order). */
+ * so far.  The pages' dispatch checks its inputs and the receive capacity
+ * (num_max_tokens_per_rank, docsearch item 10) inside its kernels; this
+ * library records such data errors in the handle on the device instead of
+ * stopping, and this call is where the caller learns of them.  Synchronises
+ * `stream`.  Returns EP_OK, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY or
+ * EP_ERR_TIMEOUT (the first set, in that order). */
 ep_status ep_handle_check(const ep_handle *handle, ep_stream_t stream);
 
 /* Size, in 32-bit words, of the fixed device scratch array ep_layout_noalloc
  * uses (128 KiB).  Every GPU that loads the library holds it until the
- * process exits. */
+ * process exits.  The library finds the array's device address on the first
+ * call on a device and again after the device's CUDA context changes (e.g.
+ * after cudaDeviceReset), so a reset device needs no action by the caller. */
 #define EP_NOALLOC_SCRATCH_WORDS (1 << 15)
 
 /* ep_layout_noalloc -- the routing layout of ep_layout, for callers that
@@ -312,14 +355,16 @@ ep_status ep_handle_check(const ep_handle *handle, ep_stream_t stream);
  * the library; a problem that needs more is rejected.  The need is
  * align4(tiles*E) + align4(tiles*R) + align4(E) + align4(tiles) + 1 words,
  * with tiles = ceil(T / tile) and tile = 128 tokens, doubled until
- * tiles*(E + R) <= 24576: every problem with E + R >= 8 fits; with very few
- * experts and millions of tokens the per-tile flags can exceed it is rejected with
- * EP_ERR_SCRATCH_LIMIT before anything is enqueued.  The first call on a
- * device looks up the array's device address (once per device, with that
- * device current); make that first call before any stream capture.  All calls
- * share the array and it keeps the last call's contents: calls whose GPU work
+ * tiles*(E + R) <= 24576.  Every problem with E + R >= 8 fits.  With very few
+ * experts and millions of tokens the one flag word per tile can push the need
+ * past the limit; such a problem is rejected with EP_ERR_SCRATCH_LIMIT before
+ * anything is enqueued.  The first call on a device looks up the array's
+ * device address (with that device current; again if the device's context
+ * changed); make that first call before any stream capture.  All calls share
+ * the array and it keeps the last call's contents: calls whose GPU work
  * overlaps (unordered streams) race on it; calls ordered on one stream do not.
- * Other limits and argument errors as for ep_layout. */
+ * EP_DEBUG logs one line per call, as for ep_layout, with the scratch words
+ * the call uses.  Other limits and argument errors as for ep_layout. */
 ep_status ep_layout_noalloc(const int32_t *topk_idx, int num_tokens, int num_topk,
                             int num_experts, int num_ranks, int expert_alignment, int capacity,
                             int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,

@@ -74,6 +74,12 @@ def test_dispatch_combine_argument_errors_on_host(L):
         assert L.ep_combine(fake, None, None, H, 0, None, None) == ep.EP_ERR_INVALID_ARG
         assert L.ep_dispatch_backward(fake, None, H, 0, None, None) == ep.EP_ERR_INVALID_ARG
         assert L.ep_combine_backward(fake, None, None, None, H, 0, None, None, None) == ep.EP_ERR_INVALID_ARG
+    # column-major FP8 dispatch: no handle, H not a multiple of 128, leading dimension below the rows
+    assert L.ep_dispatch_fp8_colmajor(None, None, 128, None, None, 64, None, None, 64, 0, None) == \
+        ep.EP_ERR_INVALID_ARG
+    for H, ld, rows, sms in ((136, 64, 64, 0), (0, 64, 64, 0), (128, 63, 64, 0), (128, 64, 64, -1)):
+        assert L.ep_dispatch_fp8_colmajor(fake, None, H, None, None, ld, None, None, rows, sms, None) == \
+            ep.EP_ERR_INVALID_ARG, (H, ld, rows, sms)
     L.ep_handle_free(None)  # no-op
     info = ep._HandleInfo()
     assert L.ep_handle_get_info(None, ctypes.byref(info)) == ep.EP_ERR_INVALID_ARG

@@ -209,3 +209,115 @@ def test_binding_refuses_buffers_the_call_would_overrun():
     valid = L.src_idx >= 0
     assert (got.cpu().numpy()[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
     assert h.check() == ep.EP_OK
+
+
+@pytest.mark.parametrize("T,num_sms,padded,ld_pad", [(2400, 0, False, 0), (2400, 16, False, 4), (2400, 0, True, 8),
+                                                     (257, 0, False, 0), (1, 0, False, 4)])
+def test_column_major_scales_through_the_token_table(T, num_sms, padded, ld_pad):
+    """ep_dispatch_fp8_colmajor (per-token scale table, then the column
+    fill): codes, column-major scales and the token table bit-exact against
+    the oracle, with unused first slots, a token with no slot, padding rows
+    and the leading dimension's slack untouched, under an SM budget and in
+    padded mode; a ragged last tile of rows (rows not a multiple of 128)."""
+    w = W.WORKLOADS["prefill"].scaled(T=T)
+    x, idx, _ = W.make_routing(w)
+    idx = idx.clone()
+    if T > 8:
+        idx[::3, 0] = -1
+        idx[5, :] = -1
+        idx[7, :2] = -1
+    C = 128 if padded else 0
+    G = w.H // 128
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R, 1, C)
+    st, L = oracle.layout(idx.numpy(), w.E, w.R, 1, C)
+    assert st == 0
+    rows = res.handle.num_recv_rows
+    ld = (rows + 3) // 4 * 4 + ld_pad
+    sc = torch.full((G, ld), -3.0, dtype=torch.float32, device=DEV)
+    recv = torch.full((rows, w.H), 0x5A, dtype=torch.uint8, device=DEV).view(torch.float8_e4m3fn)
+    tok = torch.full((T, G), -5.0, dtype=torch.float32, device=DEV)
+    src = torch.empty(rows, dtype=torch.int32, device=DEV)
+    ep.ep_dispatch_fp8_colmajor(res.handle, x.to(DEV), recv_x=recv, recv_scales=sc, token_scales=tok,
+                                recv_src_idx=src, num_sms=num_sms)
+    torch.cuda.synchronize()
+    q, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+    _, ts = oracle.quantize_rows(x)
+    valid = L.src_idx >= 0
+    got = sc.cpu().numpy()
+    assert (got[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
+    assert (got[:, :rows].T[~valid] == -3.0).all() and (got[:, rows:] == -3.0).all()
+    assert (u8(recv)[valid] == q[valid]).all() and (u8(recv)[~valid] == 0x5A).all()
+    assert (tok.cpu().numpy().view(np.uint32) == ts.view(np.uint32)).all()
+    assert (src.cpu().numpy() == L.src_idx).all()
+    assert res.handle.check() == ep.EP_OK
+
+
+def test_column_major_scales_through_the_token_table_full_size():
+    """The metric workload (group-limited gating, T=8192, H=7168, E=256,
+    R=64) at full size: every receive row's codes and every column-major
+    scale against the oracle; equal to ep_dispatch_ex's scattered form."""
+    w = W.WORKLOADS["group_limited"]
+    x, idx, _ = W.make_routing(w)
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R)
+    _, L = oracle.layout(idx.numpy(), w.E, w.R)
+    rows, G = res.handle.num_recv_rows, w.H // 128
+    xd = x.to(DEV)
+    recv, sc, tok, _ = ep.ep_dispatch_fp8_colmajor(res.handle, xd)
+    _, sc2, _ = ep.ep_dispatch_ex(res.handle, xd, True, scale_layout="col")
+    torch.cuda.synchronize()
+    assert torch.equal(sc[:, :rows], sc2[:, :rows])
+    q, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+    assert (sc[:, :rows].cpu().numpy().T.view(np.uint32) == s.view(np.uint32)).all()
+    got = recv.view(torch.uint8)
+    for r0 in range(0, rows, 8192):
+        assert (got[r0:r0 + 8192].cpu().numpy() == q[r0:r0 + 8192]).all(), r0
+    _, ts = oracle.quantize_rows(x)
+    assert (tok.cpu().numpy().view(np.uint32) == ts.view(np.uint32)).all()
+
+
+def test_column_major_token_table_argument_errors():
+    w, x, tw, res, L = setup("prefill", 64)
+    h = res.handle
+    rows, G = h.num_recv_rows, w.H // 128
+    xd = x.to(DEV)
+    with pytest.raises(ValueError, match="recv_scales"):
+        ep.ep_dispatch_fp8_colmajor(h, xd, recv_scales=torch.empty(G, rows - 1, device=DEV))
+    with pytest.raises(ValueError, match="token_scales"):
+        ep.ep_dispatch_fp8_colmajor(h, xd, token_scales=torch.empty(w.T - 1, G, device=DEV))
+    with pytest.raises(ValueError, match="H % 128"):
+        ep.ep_dispatch_fp8_colmajor(h, torch.zeros(w.T, 136, dtype=torch.bfloat16, device=DEV))
+    import ctypes
+    P = ctypes.c_void_p
+    recv = torch.empty(rows, w.H, dtype=torch.float8_e4m3fn, device=DEV)
+    sc = torch.empty(G, rows, device=DEV)
+    stream = P(torch.cuda.current_stream().cuda_stream)
+    # no token table
+    st = ep.lib().ep_dispatch_fp8_colmajor(h.ptr, P(xd.data_ptr()), w.H, P(recv.data_ptr()), P(sc.data_ptr()),
+                                           rows, None, None, rows, 0, stream)
+    assert st == ep.EP_ERR_INVALID_ARG
+    # fewer rows than the layout may use
+    tok = torch.empty(w.T, G, device=DEV)
+    st = ep.lib().ep_dispatch_fp8_colmajor(h.ptr, P(xd.data_ptr()), w.H, P(recv.data_ptr()), P(sc.data_ptr()),
+                                           rows - 1, P(tok.data_ptr()), None, rows - 1, 0, stream)
+    assert st == ep.EP_ERR_INVALID_ARG
+
+
+def test_column_major_prequantised_through_the_fill():
+    """Pre-quantised input with column-major scales takes the fill pass with
+    the input's own scale table: bit-exact, padding rows untouched."""
+    w = W.WORKLOADS["decode"]
+    x, idx, _ = W.make_routing(w)
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R, w.align, w.capacity)
+    _, L = oracle.layout(idx.numpy(), w.E, w.R, w.align, w.capacity)
+    rows, G = res.handle.num_recv_rows, w.H // 128
+    xq, xs = oracle.quantize_rows(x)
+    sc = torch.full((G, rows + 4), -3.0, device=DEV)
+    recv, sc, _ = ep.ep_dispatch_ex(res.handle, torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn), True,
+                                    x_scales=torch.from_numpy(xs).to(DEV), recv_scales=sc, scale_layout="col")
+    torch.cuda.synchronize()
+    q, s = oracle.dispatch_fp8_prequant(xq, xs, L.pos, L.n_rows)
+    valid = L.src_idx >= 0
+    got = sc.cpu().numpy()
+    assert (got[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
+    assert (got[:, :rows].T[~valid] == -3.0).all() and (got[:, rows:] == -3.0).all()
+    assert (u8(recv)[valid] == q[valid]).all()

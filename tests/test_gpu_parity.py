@@ -110,7 +110,12 @@ def test_layout_edge_cases(case):
     assert st == 0
     assert_layout_equal(res, md, L)
     assert res.handle.check() == ep.EP_OK
-    assert res.handle.layout_kernels == (1 if _one_cta_layout(T, k, E, R, C) else 2)
+    h = res.handle
+    if _one_cta_layout(T, k, E, R, C):
+        assert h.layout_path == ep.EP_LAYOUT_PATH_ONE_CTA and h.layout_kernels == 1
+    else:
+        assert h.layout_path == ep.EP_LAYOUT_PATH_TILED
+        assert h.layout_kernels == (2 if h.layout_path == ep.EP_LAYOUT_PATH_TILED else 1)
 
 
 def _one_cta_layout(T, k, E, R, C):
@@ -128,7 +133,7 @@ def test_layout_empty():
         res, md = run_layout(idx, 16, 4, 1, C)
         _, L = oracle.layout(idx.numpy(), 16, 4, 1, C)
         assert_layout_equal(res, md, L)
-        assert res.handle.layout_kernels == 1
+        assert res.handle.layout_kernels == 1 and res.handle.layout_path == ep.EP_LAYOUT_PATH_EMPTY
 
 
 def test_layout_bad_expert_id_reported():
