@@ -324,7 +324,48 @@ def cpu_baseline(w: W.Workload, seed: int, budget_s: float = 12.0, n_tok: int = 
             "sample": "%d x (layout of all %d tokens + %s dispatch and BF16 combine of the first "
                       "%d tokens), %.1f s single-threaded C" % (reps, w.T, "FP8" if w.fp8 else "BF16",
                                                                  n_tok, dt),
-            "host_cpu": host_cpu()}
+            "host_cpu": host_cpu(),
+            "all_cores": cpu_baseline_all_cores(w, x, idx, tw, y, n_tok, n_rows, budget_s / 2)}
+
+
+def cpu_baseline_all_cores(w: W.Workload, x, idx, tw, y, n_tok: int, n_rows: int, budget_s: float) -> dict:
+    """The same oracle, unchanged, over all host cores: the sample's tokens
+    split into one contiguous shard per core, each shard's dispatch and
+    combine run by its own thread (the C calls release the interpreter lock),
+    the layout (a sequential definition) on one.  A reported baseline beside
+    the single-core figure, not the target."""
+    import oracle as orc
+    from concurrent.futures import ThreadPoolExecutor
+    cores = max(1, min(os.cpu_count() or 1, n_tok))
+    bounds = [(i * n_tok // cores, (i + 1) * n_tok // cores) for i in range(cores)]
+    bounds = [(a, b) for a, b in bounds if b > a]
+    xs = [x[a:b].contiguous() for a, b in bounds]
+    ts = [np.ascontiguousarray(tw[a:b]) for a, b in bounds]
+    ys = [y[a * w.k:b * w.k].contiguous() for a, b in bounds]
+    pos = [np.arange((b - a) * w.k, dtype=np.int32).reshape(b - a, w.k) for a, b in bounds]
+
+    def shard(i):
+        n = (bounds[i][1] - bounds[i][0]) * w.k
+        if w.fp8:
+            orc.dispatch_fp8(xs[i], pos[i], n)
+        else:
+            orc.dispatch_bf16(xs[i], pos[i], n)
+        orc.combine(ys[i], ts[i], pos[i])
+
+    with ThreadPoolExecutor(max_workers=len(bounds)) as pool:
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            orc.layout(idx, w.E, w.R, w.align, w.capacity)
+            list(pool.map(shard, range(len(bounds))))
+            reps += 1
+            if time.perf_counter() - t0 > budget_s or reps >= 100:
+                break
+        dt = time.perf_counter() - t0
+    byts = oracle_bytes(w, n_tok, n_rows) * reps
+    return {"value": byts / dt / 1e9, "unit": "GB/s", "cores": len(bounds), "kind": "oracle, token-sharded",
+            "sample": "%d x (layout of all %d tokens on one thread + dispatch and combine of the first %d "
+                      "tokens in %d shards, one thread each), %.1f s" % (reps, w.T, n_tok, len(bounds), dt)}
 
 
 def host_cpu() -> str:
@@ -374,7 +415,7 @@ def run_reference(args, w):
                                        "H=7168, top-8", "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": storage_dtype(w), "data": "synthetic",
         "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample, "host_cpu": host_cpu()},
@@ -382,6 +423,13 @@ def run_reference(args, w):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def storage_dtype(w: W.Workload) -> str:
+    """The bench line's dtype: fp32 arithmetic (the FP8 scale and 448/amax,
+    the combine's fma chain), and the formats the data is stored in."""
+    disp = "e4m3 + f32 scales" if w.fp8 else "bf16"
+    return "f32 arithmetic; bf16 x -> %s dispatched; bf16 y -> bf16 combined" % disp
 
 
 def workload_config(w: W.Workload, world: int) -> dict:
@@ -522,6 +570,21 @@ def run_ours(args, w):
             last.free()
         last = h
     torch.cuda.synchronize()
+    # Combine alone, with a clean L2 (flushed and drained before each call):
+    # its in-step window also pays for writing back the dispatch's last dirty
+    # L2 lines, a fixed amount (about the L2 size) whatever the batch.
+    alone = []
+    for i in range(args.steps):
+        flush_l2()
+        torch.cuda._sleep(GPU_LEAD_CYCLES // 2)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ep.ep_combine(last, y, tw, out)
+        e1.record(stream)
+        alone.append((e0, e1))
+    torch.cuda.synchronize()
+    com_alone_ms = reduce_max(sum(a.elapsed_time(b) for a, b in alone) / len(alone), world)
     last.free()
     lay = [e[0].elapsed_time(e[1]) for e in attr]
     dis = [e[1].elapsed_time(e[2]) for e in attr]
@@ -540,7 +603,10 @@ def run_ours(args, w):
         "combine": {"us": com_ms * 1e3, "bytes": nbytes["combine"],
                     "gbs": nbytes["combine"] / (com_ms / 1e3) / 1e9},
     }
-    for kname in ("dispatch", "combine"):
+    kern["combine_clean_l2"] = {"us": com_alone_ms * 1e3, "bytes": nbytes["combine"],
+                                "gbs": nbytes["combine"] / (com_alone_ms / 1e3) / 1e9,
+                                "note": "combine alone after an L2 flush (no dirty lines of the dispatch left)"}
+    for kname in ("dispatch", "combine", "combine_clean_l2"):
         kern[kname]["frac_of_peak"] = kern[kname]["gbs"] / peak
         kern[kname]["frac_of_8tbs_nominal"] = kern[kname]["gbs"] / 8000.0
     dom = "combine" if com_ms >= dis_ms else "dispatch"
@@ -588,7 +654,7 @@ def run_ours(args, w):
             "metric": "dispatch/combine HBM GB/s & % of peak; us/call at 8192 tok, H=7168, top-8",
             "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": storage_dtype(w), "data": "synthetic",
             "config": workload_config(w, world),
             "kernels": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "decode": decode, "backward": backward, "gemm_layout": gemm_layout, "overlap": overlap,
@@ -646,6 +712,26 @@ def run_decode_latency(dev, ep, steps: int = 100) -> dict:
     d_us = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) * 1e3
     c_us = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) * 1e3
 
+    # Back to back: `steps` launches of one call inside one event pair, so the
+    # launch and event overheads of a single bracketed call drop out and what
+    # is left is the GPU time per launch (each kernel still waits for its
+    # predecessor; programmatic launch overlaps only the launch latency).
+    def back_to_back(fn):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda._sleep(GPU_LEAD_CYCLES * 12)   # ~6 ms: the host queues every launch first
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / steps
+
+    d_b2b = back_to_back(lambda: ep.ep_dispatch(h, xb, True, recv, sc))
+    c_b2b = back_to_back(lambda: ep.ep_combine(h, y, twd, out))
+    s_b2b = back_to_back(step)
+
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
@@ -669,6 +755,7 @@ def run_decode_latency(dev, ep, steps: int = 100) -> dict:
         e1.record(stream)
         torch.cuda.synchronize()
         total += e0.elapsed_time(e1)
+    g_b2b = back_to_back(graph.replay)
     status = h.check()
     del graph
     h.free()
@@ -680,6 +767,8 @@ def run_decode_latency(dev, ep, steps: int = 100) -> dict:
     return {"workload": "decode", "tokens": w.T, "hidden": w.H, "topk": w.k, "experts": w.E,
             "capacity": w.capacity, "steps": steps, "dispatch_us": d_us, "combine_us": c_us,
             "step_us_plain": d_us + c_us, "step_us_graph": total / steps * 1e3,
+            "dispatch_us_back_to_back": d_b2b, "combine_us_back_to_back": c_b2b,
+            "step_us_back_to_back": s_b2b, "step_us_graph_back_to_back": g_b2b,
             "dispatch_bytes": disp_bytes, "combine_bytes": comb_bytes}
 
 
@@ -735,11 +824,13 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
 
 
 def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> dict | None:
-    """The FP8 dispatch options that serve grouped expert GEMMs
-    (ep_dispatch_ex), on the step's layout, each timed with the L2 flushed
-    before every call: scales row-major [rows, H/128] (the step's form),
-    column-major [H/128, ld] (ld = rows rounded up to 4), and pre-quantised
-    input (e4m3 codes + row-major scales, copied unchanged)."""
+    """The FP8 dispatch options that serve grouped expert GEMMs, on the
+    step's layout, each timed with the L2 flushed before every call: scales
+    row-major [rows, H/128] (the step's form); column-major [H/128, ld]
+    (ld = rows rounded up to 4) through the per-token table and column fill
+    (ep_dispatch_fp8_colmajor) and, for comparison, with one scattered store
+    per row and group (ep_dispatch_ex); pre-quantised input (e4m3 codes +
+    scales, copied unchanged) with row-major and column-major scales."""
     if not w.fp8:
         return None
     T, H, k = w.T, w.H, w.k
@@ -776,7 +867,11 @@ def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> di
 
     row_us = timed(lambda: ep.ep_dispatch_ex(h, x_dev, True, recv_x=recv, recv_scales=sc_row))
     col_us = timed(lambda: ep.ep_dispatch_ex(h, x_dev, True, recv_x=recv, recv_scales=sc_col, scale_layout="col"))
+    tok = torch.empty(T, G, dtype=torch.float32, device=dev)
+    colt_us = timed(lambda: ep.ep_dispatch_fp8_colmajor(h, x_dev, recv_x=recv, recv_scales=sc_col, token_scales=tok))
     pq_us = timed(lambda: ep.ep_dispatch_ex(h, xq, True, x_scales=xs, recv_x=recv, recv_scales=sc_row))
+    pqc_us = timed(lambda: ep.ep_dispatch_ex(h, xq, True, x_scales=xs, recv_x=recv, recv_scales=sc_col,
+                                             scale_layout="col"))
     status = h.check()
     h.free()
     if status != ep.EP_OK:
@@ -785,8 +880,14 @@ def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> di
     q_bytes = T * H * 2 + T * k * 4 + V * H + V * G * 4
     pq_bytes = T * H + T * G * 4 + T * k * 4 + V * H + V * G * 4
     return {"scales_row_major": {"us": row_us, "bytes": q_bytes, "gbs": q_bytes / row_us / 1e3},
-            "scales_column_major": {"us": col_us, "bytes": q_bytes, "gbs": q_bytes / col_us / 1e3, "ld": ld},
-            "prequantised_input": {"us": pq_us, "bytes": pq_bytes, "gbs": pq_bytes / pq_us / 1e3}}
+            "scales_column_major_scattered": {"us": col_us, "bytes": q_bytes, "gbs": q_bytes / col_us / 1e3,
+                                              "ld": ld, "call": "ep_dispatch_ex"},
+            "scales_column_major": {"us": colt_us, "bytes": q_bytes, "gbs": q_bytes / colt_us / 1e3, "ld": ld,
+                                    "call": "ep_dispatch_fp8_colmajor (per-token table + column fill)",
+                                    "table_bytes": T * G * 4},
+            "prequantised_input": {"us": pq_us, "bytes": pq_bytes, "gbs": pq_bytes / pq_us / 1e3},
+            "prequantised_input_column_major": {"us": pqc_us, "bytes": pq_bytes, "gbs": pq_bytes / pqc_us / 1e3,
+                                                "ld": ld}}
 
 
 def run_ranks_emulated(w, dev, ep, flush_l2, worlds=(1, 8), steps: int = 10) -> dict:
@@ -862,7 +963,11 @@ def run_ranks_emulated(w, dev, ep, flush_l2, worlds=(1, 8), steps: int = 10) -> 
     return out
 
 
-NVLINK_PEER_GBS = 770.0   # measured peer copy bandwidth per direction per GPU on this machine's B200s
+# Assumed NVLink peer bandwidth per direction per GPU for the floor of the
+# cross-GPU step: a figure quoted for this GPU type's peer copies, not
+# measured by this repository (no run here has had two GPUs).  900 GB/s is
+# the nominal NVLink 5 figure.
+NVLINK_PEER_GBS = 770.0
 
 
 def run_ep_across_gpus(args, w, world, rank, local, steps: int = 10) -> dict:
@@ -936,7 +1041,7 @@ def run_ep_across_gpus(args, w, world, rank, local, steps: int = 10) -> dict:
             "nvlink_floor_ms": floor_ms,
             "frac_of_nvlink_floor": (floor_ms / ms) if ms > 0 and floor_ms > 0 else None,
             "note": "per step: layout + all-gather + plan, peer dispatch, peer combine; floor = the "
-                    "busiest rank's larger direction per phase at the measured 770 GB/s peer bandwidth"}
+                    "busiest rank's larger direction per phase at an assumed 770 GB/s peer bandwidth (not measured here)"}
 
 
 def run_overlap(w, dev, ep, idx_dev, x_dev, tw_dev, y_dev, flush_l2, reps: int = 10) -> dict:
