@@ -252,6 +252,37 @@ def test_column_major_scales_through_the_token_table(T, num_sms, padded, ld_pad)
     assert res.handle.check() == ep.EP_OK
 
 
+@pytest.mark.parametrize("H,align,num_sms", [(7168, 1, 0), (640, 1, 0), (8192 + 128, 1, 0), (7168, 4, 0),
+                                              (1024, 1, 7)])
+def test_column_major_scales_repeated_calls(H, align, num_sms):
+    """Several ep_dispatch_fp8_colmajor calls on one handle with new x each
+    time (the decode pattern), the table and scale buffers reused: every
+    call bit-exact, for 56 groups (16-byte table pieces), 5 groups (scalar
+    pieces), two chunks per token, an alignment and an SM budget."""
+    w = W.WORKLOADS["prefill"].scaled(T=777, H=H)
+    _, idx, _ = W.make_routing(w)
+    idx = idx.clone()
+    idx[::5, 1] = -1
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R, align, 0)
+    st, L = oracle.layout(idx.numpy(), w.E, w.R, align, 0)
+    assert st == 0
+    rows, G = res.handle.num_recv_rows, H // 128
+    valid = L.src_idx >= 0
+    sc = torch.full((G, rows + 4), -3.0, device=DEV)
+    tok = torch.empty(w.T, G, device=DEV)
+    for step in range(3):
+        x = W.make_x(w, 50 + step)
+        recv, sc, tok, _ = ep.ep_dispatch_fp8_colmajor(res.handle, x.to(DEV), recv_scales=sc, token_scales=tok,
+                                                       num_sms=num_sms)
+        torch.cuda.synchronize()
+        q, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+        got = sc.cpu().numpy()
+        assert (got[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all(), step
+        assert (got[:, :rows].T[~valid] == -3.0).all() and (got[:, rows:] == -3.0).all(), step
+        assert (u8(recv)[valid] == q[valid]).all(), step
+    assert res.handle.check() == ep.EP_OK
+
+
 def test_column_major_scales_through_the_token_table_full_size():
     """The metric workload (group-limited gating, T=8192, H=7168, E=256,
     R=64) at full size: every receive row's codes and every column-major
