@@ -52,3 +52,18 @@ def test_reference_arm_sample_shrinks_to_its_time_budget():
     d = json.loads(res.stdout.strip())
     assert "first 64 tokens" in d["cpu_baseline"]["sample"]
     assert d["steps"] == 20 and d["value"] > 0
+
+
+def test_cpu_baseline_reports_the_all_core_run():
+    """The CUDA arm's cpu_baseline: the single-threaded oracle (cores = 1)
+    and, beside it, the same oracle over token shards on all host threads
+    (cores = the threads it used); both on a bounded sample."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_ep_layout_10_b200 import workloads as W
+    w = W.WORKLOADS["prefill"].scaled(T=256)
+    cb = bench.cpu_baseline(w, 0, budget_s=0.2, n_tok=64)
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0
+    ac = cb["all_cores"]
+    assert ac["cores"] == min(os.cpu_count() or 1, 64) and ac["value"] > 0
+    assert "shards" in ac["sample"] and ac["unit"] == "GB/s"
