@@ -13,14 +13,17 @@
 //      histogram (shared-memory integer atomics: an integer sum does not
 //      depend on the order), token-in-rank flags, per-tile rank counts and a
 //      per-tile bad-id flag.
-//   2. layout_pos_kernel (one CTA per tile): loads the whole [tiles x E]
-//      count matrix into shared memory, derives its own tile base and the
-//      global segment offsets from it (every CTA does this redundantly: a few
-//      tens of KB from L2 per CTA instead of a serial single-CTA scan kernel),
-//      then ranks its slots in slot order with warp __match_any_sync + popc
-//      and a prefix over its warps, and writes pos[t][j] and src_idx[row].
-//      CTA 0 publishes counts, segments, rank slices, rank counts and the
-//      error word; the -1 fill of padding rows is spread over all CTAs.
+//   2. layout_pos_kernel (one CTA per tile): launched while the count
+//      kernel runs, it first counts its tile's slots per warp
+//      (__match_any_sync + popc; the ids predate the layout), then waits for
+//      the count kernel, loads the whole [tiles x E] count matrix into shared
+//      memory, derives its own tile base and the global segment offsets from
+//      it (every CTA does this redundantly: a few tens of KB from L2 per CTA
+//      instead of a serial single-CTA scan kernel), ranks its slots in slot
+//      order with a prefix over its warps, and writes pos[t][j] and
+//      src_idx[row].  CTAs 0, 1 and 2 publish the segments and error word, the
+//      expert counts, and the rank slices and counts; the -1 fill of padding
+//      rows is spread over all CTAs.
 // Both run about two tile slots per thread (256..1024 threads; the rule and
 // its measurements are in ep_internal.cuh).  The position kernel lets
 // dispatch launch only when it exits: early-launched dispatch blocks would
@@ -190,25 +193,55 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     int32_t *ids_s = wcnt + align4(W * E);               // [tile_tokens * k] when a.ids_in_smem
     __shared__ int32_t warp_s[33];
 
-#if EP_LAYOUT_POS_EARLY_TRIGGER
-    pdl_wait_then_trigger();
-#else
-    pdl_wait();
-#endif
     const int tile = blockIdx.x;
     const int t0 = tile * a.tile_tokens;
     const int nt = min(a.tile_tokens, a.T - t0);
     const int nslots = nt * a.k;
     const int64_t s0 = (int64_t)t0 * a.k;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    // The publishing is spread over up to three CTAs: CTA 0 the segments and
+    // the error word, cnt_cta the expert counts, rank_cta the rank slices and
+    // counts (it alone loads the tile rank counts).
+    const int cnt_cta = NT > 1 ? 1 : 0;
+    const int rank_cta = NT > 2 ? 2 : NT - 1;
+
+    // Before waiting for the count kernel: the tile's ids and their per-warp
+    // counts.  The ids were written before the layout began -- this kernel is
+    // launched only when every count CTA has passed its own wait, so every
+    // kernel that wrote them has completed -- and pass A touches shared memory
+    // only, so it runs while the count kernel is still working.
     if (a.ids_in_smem) load_words(ids_s, a.topk_idx + s0, nslots);
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    // A: per-expert slot counts of each warp's contiguous range of the tile's slots.
+    const int lo = (int)((int64_t)warp * nslots / W);
+    const int hi = (int)((int64_t)(warp + 1) * nslots / W);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    int32_t *my = wcnt + warp * E;
+    if (warp < W) {
+        for (int b = lo; b < hi; b += 32) {
+            const int s = b + lane;
+            const int e = (s < hi) ? tile_id(a, ids_s, s0, s) : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+            __syncwarp();
+        }
+    }
+
+#if EP_LAYOUT_POS_EARLY_TRIGGER
+    pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
     load_words(mat, a.tile_cnt, NT * E);
-    if (tile == 0) load_words(rmat, a.tile_rank, NT * R);
+    if (tile == rank_cta && a.out_rank_tok != nullptr) load_words(rmat, a.tile_rank, NT * R);
     // CTA 0 also reads every tile's bad-id flag here, so the round trip
     // overlaps the matrix load instead of delaying its publish step.
     uint32_t tile_bad = 0u;
     if (tile == 0)
         for (int t = threadIdx.x; t < NT; t += blockDim.x) tile_bad |= __ldg(a.tile_err + t);
-    for (int i = threadIdx.x; i < W * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
 
     // Tile base and total of every expert.
@@ -249,28 +282,29 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
 
     if (tile == 0) {
         for (int e = threadIdx.x; e <= E; e += blockDim.x) a.seg[e] = seg_s[e];
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            a.cnt[e] = cnt_s[e];
-            if (a.out_cnt != nullptr) a.out_cnt[e] = cnt_s[e];
-        }
-        for (int r = threadIdx.x; r <= R; r += blockDim.x) a.rank_off[r] = seg_s[r * a.epr];
-        if (a.out_rank_tok != nullptr) {
-            for (int r = threadIdx.x; r < R; r += blockDim.x) {
-                int32_t s = 0;
-                for (int t = 0; t < NT; ++t) s += rmat[t * R + r];
-                a.out_rank_tok[r] = s;
-            }
-        }
         const uint32_t bad = __syncthreads_or(tile_bad != 0u) ? kErrBadExpertId : 0u;
         // The layout (re)initialises the handle's error word.
         if (threadIdx.x == 0) *a.err = bad | (over ? kErrCapacity : 0u);
     }
+    if (tile == cnt_cta) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            a.cnt[e] = cnt_s[e];
+            if (a.out_cnt != nullptr) a.out_cnt[e] = cnt_s[e];
+        }
+    }
+    if (tile == rank_cta) {
+        for (int r = threadIdx.x; r <= R; r += blockDim.x) a.rank_off[r] = seg_s[r * a.epr];
+        if (a.out_rank_tok != nullptr) {
+            for (int r = threadIdx.x; r < R; r += blockDim.x) {
+                int32_t sum = 0;
+                for (int t = 0; t < NT; ++t) sum += rmat[t * R + r];
+                a.out_rank_tok[r] = sum;
+            }
+        }
+    }
 
     // Padding rows get src_idx = -1: each CTA takes the experts e with
     // e % ntiles == tile and a share of the rows past the last segment.
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
     for (int e = tile + NT * warp; e < E; e += NT * nwarps) {
         int32_t used = cnt_s[e];
         if (a.capacity > 0) used = min(used, a.capacity);
@@ -280,24 +314,6 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     for (int64_t row = (int64_t)seg_s[E] + (int64_t)tile * blockDim.x + threadIdx.x; row < a.n_rows;
          row += (int64_t)NT * blockDim.x)
         a.src_idx[row] = -1;
-
-    // Positions of this tile's slots.
-    const int lo = (int)((int64_t)warp * nslots / W);
-    const int hi = (int)((int64_t)(warp + 1) * nslots / W);
-    const unsigned lt_mask = (1u << lane) - 1u;
-    int32_t *my = wcnt + warp * E;
-
-    // A: per-expert slot counts of this warp's contiguous range.
-    if (warp < W) {
-        for (int b = lo; b < hi; b += 32) {
-            const int s = b + lane;
-            const int e = (s < hi) ? tile_id(a, ids_s, s0, s) : -1;
-            const unsigned peers = __match_any_sync(0xffffffffu, e);
-            if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-            __syncwarp();
-        }
-    }
-    __syncthreads();
 
     // B: exclusive prefix over the warps, starting from the tile base.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
