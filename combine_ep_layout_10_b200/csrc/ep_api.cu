@@ -178,6 +178,7 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     a.tile_threads = geo.tile_threads;
     a.ids_in_smem = geo.ids_in_smem;
     a.small = geo.small;
+    a.rank_early = 2LL * ntiles <= info.num_sms;
     a.n_rows = (int64_t)n_rows;
     a.pos = h->pos; a.src_idx = h->src_idx; a.seg = h->seg; a.rank_off = h->rank_off;
     a.cnt = h->cnt; a.tile_cnt = h->tile_cnt; a.tile_rank = h->tile_rank;

@@ -219,8 +219,9 @@ inline LayoutGeometry layout_geometry(int T, int k, int E, int R, int capacity) 
     const int pos_warps = g.tile_threads / 32;
     g.pos_warps = 12288 / E >= pos_warps ? pos_warps : (12288 / E > 0 ? 12288 / E : 1);
     const int64_t id_words = (int64_t)g.tile_tokens * k;
+    // (the position kernel keeps the slots' in-tile ranks beside the ids: twice the words)
     g.ids_in_smem = id_words <= 8192 &&
-                    layout_pos_smem_words(g.ntiles, E, R, g.pos_warps, (int)id_words) <= 50000;
+                    layout_pos_smem_words(g.ntiles, E, R, g.pos_warps, 2 * (int)id_words) <= 50000;
     const int64_t small_max = capacity > 0 ? EP_LAYOUT_SMALL_MAX_SLOTS_PADDED : EP_LAYOUT_SMALL_MAX_SLOTS;
     g.small = T > 0 && (int64_t)T * k <= small_max && E <= 512 &&
               layout_small_smem_words(T, k, E, R) <= 40000;
@@ -232,6 +233,11 @@ struct LayoutArgs {
     int T, k, E, R, epr, align, capacity;
     int tile_tokens, ntiles, sub_tokens, pos_warps, tile_threads;
     bool ids_in_smem, small;
+    // The position kernel ranks its slots inside the tile before waiting for
+    // the count kernel (with the ids in shared memory).  Only when the two
+    // kernels' CTAs need not share SMs (2 x tiles <= SMs): sharing, the extra
+    // early work slows the count kernel more than it saves (measured).
+    bool rank_early;
     int64_t n_rows;
     int32_t *pos, *src_idx, *seg, *rank_off, *cnt, *tile_cnt, *tile_rank;
     uint32_t *tile_err, *err;

@@ -191,6 +191,8 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     int32_t *seg_s = cnt_s + align4(E);                  // [E+1] segment starts
     int32_t *wcnt = seg_s + align4(E + 1);               // [W][E]
     int32_t *ids_s = wcnt + align4(W * E);               // [tile_tokens * k] when a.ids_in_smem
+    int32_t *rloc_s = ids_s + (a.ids_in_smem ? a.tile_tokens * a.k : 0);
+                                                         // [tile_tokens * k] in-tile ranks (with ids_s)
     __shared__ int32_t warp_s[33];
 
     const int tile = blockIdx.x;
@@ -227,6 +229,34 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
             __syncwarp();
+        }
+    }
+    const bool rank_early = a.ids_in_smem && a.rank_early;
+    if (rank_early) {
+        // Still before the wait: each slot's rank among the tile's slots of
+        // its expert (prefix over the warps, then the rank inside the warp),
+        // so that after the wait only the tile base and the segment start
+        // are left to add.
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int32_t run = 0;
+            for (int w = 0; w < W; ++w) {
+                const int32_t v = wcnt[w * E + e];
+                wcnt[w * E + e] = run;
+                run += v;
+            }
+        }
+        __syncthreads();
+        if (warp < W) {
+            for (int b = lo; b < hi; b += 32) {
+                const int s = b + lane;
+                const int e = (s < hi) ? tile_id(a, ids_s, s0, s) : -1;
+                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                if (e >= 0) rloc_s[s] = my[e] + __popc(peers & lt_mask);
+                __syncwarp();
+                if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+                __syncwarp();
+            }
         }
     }
 
@@ -314,6 +344,23 @@ __global__ void __launch_bounds__(kPosThreads) layout_pos_kernel(LayoutArgs a) {
     for (int64_t row = (int64_t)seg_s[E] + (int64_t)tile * blockDim.x + threadIdx.x; row < a.n_rows;
          row += (int64_t)NT * blockDim.x)
         a.src_idx[row] = -1;
+
+    if (rank_early) {
+        // position = segment start + tile base + in-tile rank, slot by slot.
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            const int e = tile_id(a, ids_s, s0, s);
+            int32_t p = -1;
+            if (e >= 0) {
+                const int32_t rel = base_s[e] + rloc_s[s];
+                if (a.capacity == 0 || rel < a.capacity) {
+                    p = seg_s[e] + rel;
+                    a.src_idx[p] = t0 + s / a.k;
+                }
+            }
+            a.pos[s0 + s] = p;
+        }
+        return;
+    }
 
     // B: exclusive prefix over the warps, starting from the tile base.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -567,8 +614,9 @@ size_t layout_count_smem(const LayoutArgs &a) {
 }
 
 size_t layout_pos_smem(const LayoutArgs &a) {
+    // with the ids in shared memory, their in-tile ranks beside them
     return (size_t)layout_pos_smem_words(a.ntiles, a.E, a.R, a.pos_warps,
-                                         a.ids_in_smem ? a.tile_tokens * a.k : 0) * 4;
+                                         a.ids_in_smem ? 2 * a.tile_tokens * a.k : 0) * 4;
 }
 
 // Raise a kernel's dynamic shared-memory limit when a launch needs more than

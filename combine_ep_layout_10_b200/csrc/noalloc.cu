@@ -147,6 +147,7 @@ extern "C" ep_status ep_layout_noalloc(const int32_t *topk_idx, int T, int k, in
     a.tile_threads = geo.tile_threads;
     a.ids_in_smem = geo.ids_in_smem;
     a.small = geo.small;
+    a.rank_early = 2LL * ntiles <= info.num_sms;
     a.n_rows = (int64_t)n_rows;
     a.pos = pos;
     a.src_idx = src_idx;
