@@ -58,9 +58,10 @@ REFERENCE_BUDGET_S = float(os.environ.get("EP_BENCH_REFERENCE_BUDGET_S", "150"))
 # DRAM traffic per launch from one ncu capture, keyed by the sha256 of the
 # kernel source it was taken on (stale -> reported as null).
 NCU_TRAFFIC = {
-    # one "ncu --set full" capture of one launch each on the metric workload
-    ("group_limited", "combine"): {"sha": "4fbe5c822556c1bf", "bytes": 940077312 + 72000512},
-    ("group_limited", "dispatch"): {"sha": "e29b25d97fe7e03a", "bytes": 117793792 + 426959104},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch each on the
+    # metric workload (one ncu capture per kernel, keyed to the kernel source)
+    ("group_limited", "combine"): {"sha": "79eb048b8ac6c125", "bytes": 940067584 + 72227328},
+    ("group_limited", "dispatch"): {"sha": "1e9e60b8fe11e2ed", "bytes": 117775872 + 425163520},
 }
 
 

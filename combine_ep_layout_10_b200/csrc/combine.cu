@@ -73,12 +73,66 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
-template <int VPT, bool LOOP, bool PEER>
+template <int VPT, bool LOOP, bool PEER, bool EARLY = false>
 __global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(CombineArgs a) {
     __shared__ const uint8_t *src_s[kMaxTopk];
     __shared__ float w_s[kMaxTopk];
-    pdl_wait_then_trigger();
     const size_t row_bytes = (size_t)a.H * 2;
+#if EP_COMBINE_POS_BEFORE_WAIT
+    // EARLY (small grids, one unit per block, local addressing): a separate
+    // instantiation, because its extra weight registers would cost the
+    // bandwidth-bound large grids resident blocks (measured: metric combine
+    // 166.8 -> 168.0 us).
+    if (EARLY && !LOOP && !PEER) {
+        // The token's k row pointers are read before the wait for the previous
+        // kernel: pos belongs to the handle and only its layout writes it, and
+        // no layout kernel lets a later kernel launch before it has finished
+        // (the count kernel, which does, writes no position), so by the time
+        // this kernel is launched the positions are complete.  The weights and
+        // the expert outputs are read only after the wait, together.
+        const int t = blockIdx.x / a.blocks_per_token;
+        const int cb = blockIdx.x - t * a.blocks_per_token;
+        if (threadIdx.x < a.k) {
+            const int p = __ldg(a.pos + (int64_t)t * a.k + threadIdx.x);
+            src_s[threadIdx.x] = p >= 0 ? a.y + (size_t)p * row_bytes : nullptr;
+        }
+        __syncthreads();
+        pdl_wait_then_trigger();
+#pragma unroll
+        for (int vi = 0; vi < VPT; ++vi) {
+            const int v = (cb * VPT + vi) * kCombineThreads + threadIdx.x;
+            if (v >= a.nvec) break;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int j0 = 0; j0 < a.k; j0 += kLoadBatch) {
+                uint4 r[kLoadBatch];
+                float wr[kLoadBatch];
+#pragma unroll
+                for (int jj = 0; jj < kLoadBatch; ++jj) {
+                    const int j = j0 + jj;
+                    const uint8_t *src = (j < a.k) ? src_s[j] : nullptr;
+                    if (src != nullptr) {
+                        r[jj] = ld_stream_v4(src + (size_t)v * 16);
+                        wr[jj] = a.w != nullptr ? __ldg(a.w + (int64_t)t * a.k + j) : 1.0f;
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < kLoadBatch; ++jj) {
+                    const int j = j0 + jj;
+                    const uint8_t *src = (j < a.k) ? src_s[j] : nullptr;
+                    if (src != nullptr) fma8(acc, wr[jj], r[jj]);
+                }
+            }
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            st_out_v4(a.out + (size_t)t * row_bytes + (size_t)v * 16, o);
+        }
+        return;
+    }
+#endif
+    pdl_wait_then_trigger();
     const int nblocks = a.T * a.blocks_per_token;  // < 2^31, checked on the host
     // One (token, vector block) pair per block unless the grid is capped
     // (LOOP): then a grid stride over the pairs.
@@ -142,6 +196,9 @@ cudaError_t launch_combine_impl(const CombineArgs &a, cudaStream_t s) {
     const bool loop = a.num_sms > 0;
     void (*kernel)(CombineArgs) = nullptr;
     if (a.vpt == 1) kernel = loop ? combine_kernel<1, true, PEER> : combine_kernel<1, false, PEER>;
+#if EP_COMBINE_POS_BEFORE_WAIT
+    if (!PEER && !loop && a.vpt == 1 && a.pos_early) kernel = combine_kernel<1, false, false, true>;
+#endif
     if (!PEER) {  // wider vectors per thread: a tuning option of the local path only
         if (a.vpt == 2) kernel = loop ? combine_kernel<2, true, false> : combine_kernel<2, false, false>;
         if (a.vpt == 4) kernel = loop ? combine_kernel<4, true, false> : combine_kernel<4, false, false>;

@@ -369,6 +369,7 @@ ep_status ep_combine_ex(const ep_handle *h, const void *y, const float *topk_w, 
     a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
     if ((int64_t)h->T * a.blocks_per_token >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.num_sms = num_sms;
+    a.pos_early = (int64_t)h->T * a.blocks_per_token <= (int64_t)EP_COMBINE_EARLY_MAX_BLOCKS_PER_SM * info.num_sms;
     if (debug_enabled())
         std::fprintf(stderr, "ep: combine T=%d H=%d blocks=%lld num_sms=%d\n", h->T, H,
                      (long long)h->T * a.blocks_per_token, num_sms);
@@ -402,6 +403,7 @@ ep_status ep_dispatch_backward(const ep_handle *h, const void *grad_recv, int H,
     a.blocks_per_token = (a.nvec + EP_COMBINE_THREADS * a.vpt - 1) / (EP_COMBINE_THREADS * a.vpt);
     if ((int64_t)h->T * a.blocks_per_token >= ((int64_t)1 << 31)) return EP_ERR_INVALID_ARG;
     a.num_sms = 0;
+    a.pos_early = (int64_t)h->T * a.blocks_per_token <= (int64_t)EP_COMBINE_EARLY_MAX_BLOCKS_PER_SM * info.num_sms;
     return cuda_status(launch_combine(a, stream));
 }
 

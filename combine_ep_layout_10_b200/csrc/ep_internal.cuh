@@ -32,6 +32,12 @@
 #ifndef EP_COMBINE_VPT            // combine: 16-byte vectors per thread (1, 2 or 4)
 #define EP_COMBINE_VPT 1
 #endif
+#ifndef EP_COMBINE_POS_BEFORE_WAIT  // combine (local, one unit per block, small grids) reads the token's
+#define EP_COMBINE_POS_BEFORE_WAIT 1  // positions before its programmatic wait (the layout kernels then signal at exit)
+#endif
+#ifndef EP_COMBINE_EARLY_MAX_BLOCKS_PER_SM  // ... small grid: at most this many blocks per SM
+#define EP_COMBINE_EARLY_MAX_BLOCKS_PER_SM 8
+#endif
 #ifndef EP_COMBINE_L2_PREFETCH    // combine: add the .L2::256B prefetch hint to the row loads
 #define EP_COMBINE_L2_PREFETCH 0
 #endif
@@ -83,6 +89,9 @@
 #endif
 #ifndef EP_DISPATCH_EARLY_TRIGGER    // dispatch kernels let their dependents launch at their start
 #define EP_DISPATCH_EARLY_TRIGGER 1
+#endif
+#if EP_COMBINE_POS_BEFORE_WAIT && EP_LAYOUT_POS_EARLY_TRIGGER
+#error "the combine reads positions before its wait: the position kernel must signal at its exit"
 #endif
 #ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
 #define EP_USE_PDL 1
@@ -304,6 +313,7 @@ struct CombineArgs {
     int vpt;                 // vectors per thread: 1, 2 or 4
     int blocks_per_token;    // ceil(nvec / (128 * vpt))
     int num_sms;             // 0: one block per (token, vector block); else grid capped
+    bool pos_early;          // small grid: read the positions before the programmatic wait
     // Multi-rank (peer) addressing, used instead of pos / y:
     const int2 *src;                 // [T, k] (rank, row) of each slot's expert output, rank -1 if none
     const uint8_t *const *peer_y;    // [world] device pointers to every rank's expert outputs

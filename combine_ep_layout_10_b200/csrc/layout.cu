@@ -446,9 +446,19 @@ __device__ void small_fill_padding_tails(const LayoutArgs &a, int32_t *cnt_h) {
     }
 }
 
+// Kernels that write positions let their dependents launch only at their
+// exit when the combine reads positions before its own wait.
+__device__ __forceinline__ void layout_writer_wait() {
+#if EP_COMBINE_POS_BEFORE_WAIT
+    pdl_wait();
+#else
+    pdl_wait_then_trigger();
+#endif
+}
+
 __global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
-    pdl_wait_then_trigger();
+    layout_writer_wait();
     if (blockIdx.x > 0) {  // padding helper (padded mode only)
         small_fill_padding_tails(a, reinterpret_cast<int32_t *>(smem));
         return;
@@ -587,7 +597,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutArgs 
 // T == 0: no tiles; one CTA writes the (empty or padded) segments, zero
 // counts, -1 over every row and a clear error word.
 __global__ void __launch_bounds__(kPosThreads) layout_empty_kernel(LayoutArgs a) {
-    pdl_wait_then_trigger();
+    layout_writer_wait();
     for (int e = threadIdx.x; e <= a.E; e += blockDim.x)
         a.seg[e] = a.capacity > 0 ? e * a.capacity : 0;
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
