@@ -153,7 +153,6 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
     h->experts_per_rank = E / R;
     h->tile_tokens = geo.tile_tokens;
     h->ntiles = ntiles;
-
     h->n_rows = (int64_t)n_rows;
     h->device = dev;
     h->stream = stream;
@@ -193,8 +192,7 @@ ep_status ep_layout(const int32_t *topk_idx, int T, int k, int E, int R, int A, 
         std::fprintf(stderr,
                      "ep: layout T=%d k=%d E=%d R=%d align=%d capacity=%d rows=%lld path=%s tiles=%d "
                      "tile_tokens=%d threads=%d\n",
-                     T, k, E, R, A, C, (long long)n_rows,
-                     geo.small ? "one-cta" : "tiled", geo.ntiles,
+                     T, k, E, R, A, C, (long long)n_rows, geo.small ? "one-cta" : "tiled", geo.ntiles,
                      geo.tile_tokens, geo.small ? 1024 : geo.tile_threads);
     e = launch_layout(a, stream);  // also (re)initialises the error word
     if (e != cudaSuccess) {
