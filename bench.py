@@ -598,7 +598,10 @@ def run_ours(args, w):
     peak = peaks["hbm_gbs"]
     kern = {
         "note": "per-call windows from an attribution pass of the same steps",
-        "layout": {"us": lay_ms * 1e3, "bytes": nbytes["layout"], "launches_per_step": layout_kernels},
+        "layout": {"us": lay_ms * 1e3, "bytes": nbytes["layout"], "launches_per_step": layout_kernels,
+                   "share_of_step_us": (step_ms - dis_ms - com_ms) * 1e3,
+                   "share_note": "step minus the dispatch and combine windows: what the layout adds to a "
+                                 "step with no events between its kernels"},
         "dispatch": {"us": dis_ms * 1e3, "bytes": nbytes["dispatch"],
                      "gbs": nbytes["dispatch"] / (dis_ms / 1e3) / 1e9},
         "combine": {"us": com_ms * 1e3, "bytes": nbytes["combine"],
