@@ -635,7 +635,7 @@ def run_ours(args, w):
 
     gemm_layout = None
     if not args.no_gemm_layout:
-        gemm_layout = run_gemm_layout(w, dev, ep, idx, x, flush_l2)
+        gemm_layout = run_gemm_layout(w, dev, ep, idx, x, flush_l2, y=y, tw=tw)
 
     overlap = None
     if not args.no_overlap:
@@ -827,14 +827,21 @@ def run_backward(w, dev, ep, idx_dev, tw_dev, y_dev, flush_l2, steps: int = 20) 
             "dispatch_topk": {"us": t_us, "bytes": t_bytes, "note": "latency-bound (~1.6 MB)"}}
 
 
-def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> dict | None:
+def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20, y=None, tw=None) -> dict | None:
     """The FP8 dispatch options that serve grouped expert GEMMs, on the
     step's layout, each timed with the L2 flushed before every call: scales
     row-major [rows, H/128] (the step's form); column-major [H/128, ld]
     (ld = rows rounded up to 4) through the per-token table and column fill
     (ep_dispatch_fp8_colmajor) and, for comparison, with one scattered store
     per row and group (ep_dispatch_ex); pre-quantised input (e4m3 codes +
-    scales, copied unchanged) with row-major and column-major scales."""
+    scales, copied unchanged) with row-major and column-major scales.
+
+    With y and tw, also each of the two quantising forms followed by the
+    step's combine in one window (`in_step`): a dispatch leaves L2 full of
+    dirty lines whose write-back the next kernel pays for, and the column
+    fill, run right after the dispatch, pays part of that inside its own
+    window; the difference of the two windows is what the column-major
+    form adds to a step."""
     if not w.fp8:
         return None
     T, H, k = w.T, w.H, w.k
@@ -876,6 +883,17 @@ def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> di
     pq_us = timed(lambda: ep.ep_dispatch_ex(h, xq, True, x_scales=xs, recv_x=recv, recv_scales=sc_row))
     pqc_us = timed(lambda: ep.ep_dispatch_ex(h, xq, True, x_scales=xs, recv_x=recv, recv_scales=sc_col,
                                              scale_layout="col"))
+    in_step = None
+    if y is not None and tw is not None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        row_c = timed(lambda: (ep.ep_dispatch_ex(h, x_dev, True, recv_x=recv, recv_scales=sc_row),
+                               ep.ep_combine(h, y, tw, out)))
+        col_c = timed(lambda: (ep.ep_dispatch_fp8_colmajor(h, x_dev, recv_x=recv, recv_scales=sc_col,
+                                                           token_scales=tok),
+                               ep.ep_combine(h, y, tw, out)))
+        in_step = {"row_major_then_combine_us": row_c, "column_major_then_combine_us": col_c,
+                   "column_major_adds_us": col_c - row_c,
+                   "column_major_equivalent_us": row_us + col_c - row_c}
     status = h.check()
     h.free()
     if status != ep.EP_OK:
@@ -891,7 +909,9 @@ def run_gemm_layout(w, dev, ep, idx_dev, x_dev, flush_l2, steps: int = 20) -> di
                                     "table_bytes": T * G * 4},
             "prequantised_input": {"us": pq_us, "bytes": pq_bytes, "gbs": pq_bytes / pq_us / 1e3},
             "prequantised_input_column_major": {"us": pqc_us, "bytes": pq_bytes, "gbs": pq_bytes / pqc_us / 1e3,
-                                                "ld": ld}}
+                                                "ld": ld},
+            "in_step": None if in_step is None else dict(
+                in_step, column_major_equivalent_gbs=q_bytes / in_step["column_major_equivalent_us"] / 1e3)}
 
 
 def run_ranks_emulated(w, dev, ep, flush_l2, worlds=(1, 8), steps: int = 10) -> dict:

@@ -301,31 +301,37 @@ cudaError_t launch_dispatch_impl(const DispatchArgs &a, cudaStream_t st) {
 // floats; 16-byte loads when rows allow, all of a thread's loads issued
 // before any is used, so a tile costs about one memory round trip) into
 // shared memory and then stores every group's column of the tile as one
-// contiguous run of up to kFillRows floats.  The table is read with an
-// evict-first L2 policy: each entry is dead once its rows are filled.
+// contiguous run of up to kFillRows floats.
+// Behind the quantising dispatch the pass is bound by what that kernel
+// leaves behind, not by its own work (measured, metric workload, with
+// per-block timestamps): its blocks are released about 0.9 us after the
+// dispatch's last block has issued its stores, the one gather round trip
+// then takes 1.6-4.1 us (median 2.4) and issuing the column stores 2.0-3.2 us
+// (median 2.8), because L2 is full of the dispatch's dirty code lines and
+// every new line waits for one to be written back; neither an all-hit table
+// (every row reading one of 64 tokens) nor dropping the stores' DRAM
+// traffic changed the call's time.
 constexpr int kFillRows = 128;
 constexpr int kFillGroups = 64;
 constexpr int kFillThreads = 256;
 constexpr int kFillVecPerThread = kFillRows / (2 * (kFillThreads / 32));  // rows of a thread in the 16-byte gather
 static_assert(kFillGroups / 4 <= 16, "a half-warp holds one row's 16-byte pieces");
 
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-__device__ __forceinline__ float4 ld_table_v4(const float *p, uint64_t pol) {
+// Table loads use the default L2 policy: every entry is read once per
+// receive row of its token (k times), so it should stay (measured: an
+// evict-first policy here cost the pre-quantised column-major call about
+// 0.5 us; evict-last and evict-unchanged were no better than the default).
+__device__ __forceinline__ float4 ld_table_v4(const float *p) {
     float4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-                 : "l"(p), "l"(pol));
+                 : "l"(p));
     return r;
 }
 
-__device__ __forceinline__ float ld_table(const float *p, uint64_t pol) {
+__device__ __forceinline__ float ld_table(const float *p) {
     float r;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(r) : "l"(p), "l"(pol));
+    asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(r) : "l"(p));
     return r;
 }
 
@@ -339,14 +345,17 @@ __global__ void __launch_bounds__(kFillThreads) scale_fill_kernel(ScaleFillArgs 
     const int64_t ntiles = (a.n_rows + kFillRows - 1) / kFillRows;
     // The source tokens of the first tile are read before the wait for the
     // dispatch: the layout wrote them, and it completed before the dispatch
-    // (this kernel's predecessor) began.  The table is read only after it.
+    // (this kernel's predecessor) began.  The table is read only after it,
+    // unless it is the caller's input (then there is no wait here at all).
     if (blockIdx.x < ntiles) {
         const int64_t p0 = (int64_t)blockIdx.x * kFillRows;
         const int n = (int)min((int64_t)kFillRows, a.n_rows - p0);
         for (int i = tid; i < n; i += kFillThreads) src_s[i] = __ldg(a.src_idx + p0 + i);
     }
-    pdl_wait_then_trigger();
-    const uint64_t pol = l2_evict_first_policy();
+    if (a.table_is_input)
+        pdl_trigger();  // nothing this pass reads or writes is touched by the copy kernel
+    else
+        pdl_wait_then_trigger();
     const int g0 = blockIdx.y * kFillGroups;
     const int gn = min(kFillGroups, a.G - g0);
     const int ldt = gn | 1;  // odd row stride: the column reads below hit distinct banks
@@ -369,7 +378,7 @@ __global__ void __launch_bounds__(kFillThreads) scale_fill_kernel(ScaleFillArgs 
                 v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (i < n && c < gv) {
                     const int32_t t = src_s[i];
-                    if (t >= 0) v[q] = ld_table_v4(a.table + (int64_t)t * a.G + g0 + 4 * c, pol);
+                    if (t >= 0) v[q] = ld_table_v4(a.table + (int64_t)t * a.G + g0 + 4 * c);
                 }
             }
 #pragma unroll
@@ -390,7 +399,7 @@ __global__ void __launch_bounds__(kFillThreads) scale_fill_kernel(ScaleFillArgs 
 #pragma unroll
                 for (int h = 0; h < kFillGroups; h += 32) {
                     const int g = h + lane;
-                    if (g < gn) tile_s[i * ldt + g] = t >= 0 ? ld_table(a.table + (int64_t)t * a.G + g0 + g, pol) : 0.0f;
+                    if (g < gn) tile_s[i * ldt + g] = t >= 0 ? ld_table(a.table + (int64_t)t * a.G + g0 + g) : 0.0f;
                 }
             }
         }
@@ -406,6 +415,9 @@ __global__ void __launch_bounds__(kFillThreads) scale_fill_kernel(ScaleFillArgs 
         }
         __syncthreads();  // src_s / tile_s are rewritten by the next tile
     }
+    // Started early: complete only after the copy kernel has, so that what
+    // follows in the stream sees both.
+    if (a.table_is_input) pdl_wait();
 }
 
 }  // namespace
@@ -416,6 +428,7 @@ cudaError_t launch_scale_fill(const ScaleFillArgs &a, cudaStream_t st) {
     if (a.n_rows == 0 || a.G == 0) return cudaSuccess;
     if (a.vec_in && (a.G % 4 != 0 || (reinterpret_cast<uintptr_t>(a.table) & 15u) != 0))
         return cudaErrorInvalidValue;
+    if (a.table_is_input && a.num_sms > 0) return cudaErrorInvalidValue;
     const int64_t ntiles = (a.n_rows + kFillRows - 1) / kFillRows;
     const int gchunks = (a.G + kFillGroups - 1) / kFillGroups;
     int64_t grid = ntiles;

@@ -272,6 +272,10 @@ ep_status ep_dispatch_ex(const ep_handle *h, const void *x, const float *x_scale
         f.G = (int)G;
         f.num_sms = num_sms;
         f.vec_in = G % 4 == 0 && aligned(x_scales, 16);
+        // Without an SM budget the pass starts in the copy kernel's last wave:
+        // the input table predates it (with a budget its blocks would wait on
+        // SMs the caller left to other work).
+        f.table_is_input = EP_FILL_EARLY_START && num_sms == 0;
         e = launch_scale_fill(f, stream);
     }
     if (e == cudaSuccess && recv_src_idx != nullptr && h->n_rows > 0)

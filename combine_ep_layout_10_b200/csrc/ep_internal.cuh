@@ -93,6 +93,9 @@
 #if EP_COMBINE_POS_BEFORE_WAIT && EP_LAYOUT_POS_EARLY_TRIGGER
 #error "the combine reads positions before its wait: the position kernel must signal at its exit"
 #endif
+#ifndef EP_FILL_EARLY_START          // fill pass from an input table starts before the copy kernel completes
+#define EP_FILL_EARLY_START 1
+#endif
 #ifndef EP_USE_PDL                // launch kernels with programmatic dependent launch
 #define EP_USE_PDL 1
 #endif
@@ -112,6 +115,12 @@ namespace ep {
 __device__ __forceinline__ void pdl_wait() {
 #if EP_USE_PDL
     asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+#if EP_USE_PDL
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #endif
 }
 
@@ -301,6 +310,11 @@ struct ScaleFillArgs {
     int G;                   // H / 128
     int num_sms;             // 0: one block per tile; else grid capped
     bool vec_in;             // table rows read as 16-byte vectors (G % 4 == 0, table 16-byte aligned)
+    // The table is the caller's input (pre-quantised scales), written before
+    // the copy kernel this pass follows began, which writes no scale: the
+    // pass starts without waiting for it, and waits only before it exits, so
+    // that this grid completes after the copy kernel.  Not with num_sms.
+    bool table_is_input;
 };
 
 struct CombineArgs {

@@ -2,7 +2,9 @@
 
 * pre-quantised FP8 input (codes + scales) is copied bit-exactly;
 * a column-major scale layout holds exactly the row-major scales, transposed;
-* an SM budget (num_sms) changes the launch shape, never the result.
+* an SM budget (num_sms) changes the launch shape, never the result;
+* the column-major fill pass is exact on back-to-back calls and graph
+  replays, also where it starts before the kernel it follows completes.
 """
 import numpy as np
 import pytest
@@ -352,3 +354,76 @@ def test_column_major_prequantised_through_the_fill():
     assert (got[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all()
     assert (got[:, :rows].T[~valid] == -3.0).all() and (got[:, rows:] == -3.0).all()
     assert (u8(recv)[valid] == q[valid]).all()
+
+
+
+@pytest.mark.parametrize("prequant", [False, True])
+def test_column_major_back_to_back_calls_and_graph_replays(prequant):
+    """Column-major scales through the fill pass, four calls enqueued back to
+    back on one handle (new x each, one shared token table for the quantising
+    call, no synchronisation in between) and three replays of a captured call
+    (new x copied in before each, results copied out after each, one
+    synchronisation at the end): each bit-exact.  With pre-quantised input the
+    fill pass starts before the copy kernel completes (its table is the
+    input), so this also checks that it never runs ahead of what it needs."""
+    w = W.WORKLOADS["prefill"].scaled(T=1500)
+    _, idx, _ = W.make_routing(w)
+    res = ep.ep_layout(idx.to(DEV), w.E, w.R)
+    st, L = oracle.layout(idx.numpy(), w.E, w.R)
+    assert st == 0
+    h = res.handle
+    rows, G = h.num_recv_rows, w.H // 128
+    valid = L.src_idx >= 0
+    xs = [W.make_x(w, 90 + i) for i in range(4)]
+    if prequant:
+        qs = [oracle.quantize_rows(x) for x in xs]
+        ins = [(torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn), torch.from_numpy(xsc).to(DEV))
+               for xq, xsc in qs]
+    else:
+        ins = [(x.to(DEV), None) for x in xs]
+    tok = torch.empty(w.T, G, device=DEV)
+
+    def call(xin, sin, recv=None, sc=None):
+        if prequant:
+            return ep.ep_dispatch_ex(h, xin, True, x_scales=sin, recv_x=recv, recv_scales=sc, scale_layout="col")[:2]
+        return ep.ep_dispatch_fp8_colmajor(h, xin, recv_x=recv, recv_scales=sc, token_scales=tok)[:2]
+
+    def check(i, recv, sc, what):
+        if prequant:
+            q, s = oracle.dispatch_fp8_prequant(qs[i][0], qs[i][1], L.pos, L.n_rows)
+        else:
+            q, s = oracle.dispatch_fp8(xs[i], L.pos, L.n_rows)
+        assert (sc.cpu().numpy()[:, :rows].T[valid].view(np.uint32) == s[valid].view(np.uint32)).all(), what
+        assert (u8(recv)[valid] == q[valid]).all(), what
+
+    torch.cuda.synchronize()
+    outs = [call(xin, sin) for xin, sin in ins]
+    torch.cuda.synchronize()
+    for i, (recv, sc) in enumerate(outs):
+        check(i, recv, sc, ("back to back", i))
+
+    xin = torch.empty_like(ins[0][0])
+    sin = torch.empty_like(ins[0][1]) if prequant else None
+    recv = torch.empty(rows, w.H, dtype=torch.float8_e4m3fn, device=DEV)
+    sc = torch.empty(G, (rows + 3) // 4 * 4, device=DEV)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        call(xin, sin, recv, sc)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        call(xin, sin, recv, sc)
+    snaps = []
+    for xi, si in ins[:3]:
+        xin.copy_(xi)
+        if prequant:
+            sin.copy_(si)
+        graph.replay()
+        snaps.append((recv.clone(), sc.clone()))
+    torch.cuda.synchronize()
+    for i, (r, s) in enumerate(snaps):
+        check(i, r, s, ("replay", i))
+    assert h.check() == ep.EP_OK
+    del graph
