@@ -61,7 +61,7 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch each on the
     # metric workload (one ncu capture per kernel, keyed to the kernel source)
     ("group_limited", "combine"): {"sha": "79eb048b8ac6c125", "bytes": 940067584 + 72227328},
-    ("group_limited", "dispatch"): {"sha": "1e9e60b8fe11e2ed", "bytes": 117775872 + 425163520},
+    ("group_limited", "dispatch"): {"sha": "aa2ecec9c00a91c0", "bytes": 117774848 + 425984768},
 }
 
 

@@ -1,6 +1,6 @@
 """EP_DEBUG host logging (GPU): one stderr line per layout / dispatch /
-combine / no-allocation layout call with the launch shape the library chose;
-silent by default."""
+column-major dispatch / combine / no-allocation layout call with the launch
+shape the library chose; silent by default."""
 import os
 import subprocess
 import sys
@@ -22,6 +22,8 @@ for name, T in (("tiny", 128), ("prefill", 512)):
     res = ep.ep_layout(idx.cuda(), w.E, w.R)
     recv, sc, _ = ep.ep_dispatch(res.handle, x.cuda(), w.fp8)
     out = ep.ep_combine(res.handle, torch.zeros(res.handle.num_recv_rows, w.H, dtype=torch.bfloat16, device="cuda"), tw.cuda())
+    if name == "prefill":
+        ep.ep_dispatch_fp8_colmajor(res.handle, x.cuda())
     torch.cuda.synchronize()
     res.handle.free()
 w = W.WORKLOADS["prefill"].scaled(T=512)
@@ -52,7 +54,9 @@ def test_debug_log_lines():
     noalloc = [ln for ln in lines if ln.startswith("ep: layout_noalloc ")]
     assert len(noalloc) == 1
     assert "path=tiled" in noalloc[0] and "scratch_words=" in noalloc[0] and "of 32768" in noalloc[0]
-    assert sum(ln.startswith("ep: dispatch") for ln in lines) == 2
+    assert sum(ln.startswith("ep: dispatch ") for ln in lines) == 2
+    colmajor = [ln for ln in lines if ln.startswith("ep: dispatch_fp8_colmajor ")]
+    assert len(colmajor) == 1 and "T=512" in colmajor[0] and "ld=4096" in colmajor[0]
     assert sum(ln.startswith("ep: combine") for ln in lines) == 2
     layouts = [ln for ln in lines if ln.startswith("ep: layout ")]
     assert "path=one-cta" in layouts[0]                     # tiny: 128 tokens x 4 slots = 512 slots
