@@ -187,6 +187,98 @@ __global__ void __launch_bounds__(kCombineThreads, LOOP ? 8 : 1) combine_kernel(
     }
 }
 
+// Row pointer and weight of slot j of token t (thread j < k of a unit).
+template <bool PEER>
+__device__ __forceinline__ void combine_slot(const CombineArgs &a, int t, int j, size_t row_bytes,
+                                             const uint8_t *&src, float &wt) {
+    const int64_t s = (int64_t)t * a.k + j;
+    src = nullptr;
+    if (PEER) {
+        const int2 d = __ldg(a.src + s);
+        if (d.x >= 0) src = a.peer_y[d.x] + (size_t)d.y * row_bytes;
+    } else {
+        const int p = __ldg(a.pos + s);
+        if (p >= 0) src = a.y + (size_t)p * row_bytes;
+    }
+    wt = a.w != nullptr ? __ldg(a.w + s) : 1.0f;
+}
+
+// The grid-capped form (an SM budget): a block walks the (token, vector
+// block) units with a grid stride, one vector per thread, and the next
+// unit's row pointers and weights are loaded (threads j < k) before this
+// unit's row loads are issued and published to the other half of a double
+// buffer after them, so that a unit costs one memory round trip, not two.
+// Same arithmetic as combine_kernel.
+template <bool PEER>
+__global__ void __launch_bounds__(kCombineThreads, 8) combine_loop_kernel(CombineArgs a) {
+    __shared__ const uint8_t *src_s[2][kMaxTopk];
+    __shared__ float w_s[2][kMaxTopk];
+    const size_t row_bytes = (size_t)a.H * 2;
+    pdl_wait_then_trigger();
+    const int nblocks = a.T * a.blocks_per_token;  // < 2^31, checked on the host
+    const int tid = threadIdx.x;
+    int b = blockIdx.x;
+    if (b >= nblocks) return;
+    if (tid < a.k) {
+        const uint8_t *src;
+        float wt;
+        combine_slot<PEER>(a, b / a.blocks_per_token, tid, row_bytes, src, wt);
+        src_s[0][tid] = src;
+        w_s[0][tid] = wt;
+    }
+    int cur = 0;
+#pragma unroll 1
+    for (; b < nblocks; b += gridDim.x) {
+        __syncthreads();  // buffer cur is published; nobody reads buffer cur ^ 1 any more
+        // The next unit's slot: only the loads here; the pointer is formed
+        // after this unit's row loads, so nothing waits on them early.
+        const int bn = b + gridDim.x;
+        int2 nd = make_int2(-1, -1);  // (rank, row) of the slot; rank 0 when local
+        float nw = 0.0f;
+        if (tid < a.k && bn < nblocks) {
+            const int64_t s = (int64_t)(bn / a.blocks_per_token) * a.k + tid;
+            if (PEER)
+                nd = __ldg(a.src + s);
+            else
+                nd = make_int2(0, __ldg(a.pos + s));
+            nw = a.w != nullptr ? __ldg(a.w + s) : 1.0f;
+        }
+        const int t = b / a.blocks_per_token;
+        const int cb = b - t * a.blocks_per_token;
+        const int v = cb * kCombineThreads + tid;
+        if (v < a.nvec) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int j0 = 0; j0 < a.k; j0 += kLoadBatch) {
+                uint4 r[kLoadBatch];
+#pragma unroll
+                for (int jj = 0; jj < kLoadBatch; ++jj) {
+                    const int j = j0 + jj;
+                    const uint8_t *src = (j < a.k) ? src_s[cur][j] : nullptr;
+                    if (src != nullptr) r[jj] = ld_stream_v4(src + (size_t)v * 16);
+                }
+#pragma unroll
+                for (int jj = 0; jj < kLoadBatch; ++jj) {
+                    const int j = j0 + jj;
+                    const uint8_t *src = (j < a.k) ? src_s[cur][j] : nullptr;
+                    if (src != nullptr) fma8(acc, w_s[cur][j], r[jj]);
+                }
+            }
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            st_out_v4(a.out + (size_t)t * row_bytes + (size_t)v * 16, o);
+        }
+        if (tid < a.k) {
+            const bool ok = PEER ? nd.x >= 0 : nd.y >= 0;
+            src_s[cur ^ 1][tid] = !ok ? nullptr : (PEER ? a.peer_y[nd.x] : a.y) + (size_t)nd.y * row_bytes;
+            w_s[cur ^ 1][tid] = nw;
+        }
+        cur ^= 1;
+    }
+}
+
 template <bool PEER>
 cudaError_t launch_combine_impl(const CombineArgs &a, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
@@ -195,7 +287,7 @@ cudaError_t launch_combine_impl(const CombineArgs &a, cudaStream_t s) {
         return cudaErrorInvalidConfiguration;
     const bool loop = a.num_sms > 0;
     void (*kernel)(CombineArgs) = nullptr;
-    if (a.vpt == 1) kernel = loop ? combine_kernel<1, true, PEER> : combine_kernel<1, false, PEER>;
+    if (a.vpt == 1) kernel = loop ? combine_loop_kernel<PEER> : combine_kernel<1, false, PEER>;
 #if EP_COMBINE_POS_BEFORE_WAIT
     if (!PEER && !loop && a.vpt == 1 && a.pos_early) kernel = combine_kernel<1, false, false, true>;
 #endif

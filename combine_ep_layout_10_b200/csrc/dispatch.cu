@@ -190,6 +190,129 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
     }
 }
 
+// The 16 e4m3 codes of a thread's channels given its group's 448 / amax
+// (RNE-satfinite e4m3 of the correctly rounded product), as in
+// dispatch_fp8_kernel.
+__device__ __forceinline__ uint4 e4m3_codes16(const float *f, float inv) {
+    uint32_t b[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float2 pr = make_float2(__fmul_rn(f[2 * q], inv), __fmul_rn(f[2 * q + 1], inv));
+        b[q] = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
+    }
+    return make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
+}
+
+// The grid-capped form (an SM budget) of dispatch_fp8_kernel: a block walks
+// the units with a grid stride, and as soon as a unit's codes are made the
+// next unit's x vectors and row positions are loaded, so that their round
+// trip overlaps this unit's stores; the next unit's row pointers go to the
+// other half of a double buffer.  Same arithmetic as dispatch_fp8_kernel.
+template <bool PEER>
+__global__ void __launch_bounds__(512) dispatch_fp8_loop_kernel(DispatchArgs a) {
+    __shared__ uint8_t *row_s[2][kMaxTopk];
+    __shared__ float *srow_s[2][kMaxTopk];
+    __shared__ float *tok_s[2];  // the unit's token row of the per-token scale table, or nullptr
+#if EP_DISPATCH_EARLY_TRIGGER
+    pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
+    const int tid = threadIdx.x;
+    const bool leader = (tid & 7) == 0;
+    const int G = a.H / 128;
+    int u = blockIdx.x;
+    if (u >= a.nunits) return;
+    uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+    {
+        const int t = u / a.nchunks;
+        const int ch0 = (u - t * a.nchunks) * a.chunk;
+        if (tid * 16 < min(a.chunk, a.H - ch0)) {
+            const uint8_t *src = a.x + ((int64_t)t * a.H + ch0 + tid * 16) * 2;
+            v0 = ld_nc_v4(src);
+            v1 = ld_nc_v4(src + 16);
+        }
+        slot_rows<PEER>(a, t, (size_t)a.H, row_s[0], srow_s[0]);
+        if (tid == 0) tok_s[0] = a.tok_scales != nullptr ? a.tok_scales + (int64_t)t * G : nullptr;
+    }
+    int cur = 0;
+#pragma unroll 1
+    for (; u < a.nunits; u += gridDim.x) {
+        __syncthreads();  // buffer cur is published; nobody reads buffer cur ^ 1 any more
+        const int t = u / a.nchunks;
+        const int ch0 = (u - t * a.nchunks) * a.chunk;
+        const int chn = min(a.chunk, a.H - ch0);
+        const int ch = ch0 + tid * 16;
+        const bool act = tid * 16 < chn;
+        float f[16];
+        unpack8(v0, f);
+        unpack8(v1, f + 8);
+        float amax = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(f[q]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        uint4 q16 = make_uint4(0u, 0u, 0u, 0u);
+        float scale = 0.0f;
+        if (act && amax != 0.0f) {
+            scale = __fdiv_rn(amax, 448.0f);
+            q16 = e4m3_codes16(f, __fdiv_rn(448.0f, amax));
+        }
+        // The next unit's loads, issued before this unit's stores.
+        const int un = u + gridDim.x;
+        const bool more = un < a.nunits;
+        const int tn = more ? un / a.nchunks : 0;
+        v0 = make_uint4(0u, 0u, 0u, 0u);
+        v1 = v0;
+        int np = -1;
+        int2 nd = make_int2(-1, -1);
+        if (more) {
+            const int nch0 = (un - tn * a.nchunks) * a.chunk;
+            if (tid * 16 < min(a.chunk, a.H - nch0)) {
+                const uint8_t *src = a.x + ((int64_t)tn * a.H + nch0 + tid * 16) * 2;
+                v0 = ld_nc_v4(src);
+                v1 = ld_nc_v4(src + 16);
+            }
+            if (tid < a.k) {
+                if (PEER)
+                    nd = __ldg(a.dst + (int64_t)tn * a.k + tid);
+                else
+                    np = __ldg(a.pos + (int64_t)tn * a.k + tid);
+            }
+        }
+        if (act) {
+            const int g = ch / 128;
+            if (leader && tok_s[cur] != nullptr) st_table_keep(tok_s[cur] + g, scale);
+            for (int j = 0; j < a.k; ++j) {
+                uint8_t *row = row_s[cur][j];
+                if (row == nullptr) continue;
+                st_row_v4(row + ch, q16);
+                if (leader && srow_s[cur][j] != nullptr) srow_s[cur][j][(int64_t)g * a.s_grp] = scale;
+            }
+        }
+        if (more) {
+            if (tid < a.k) {
+                uint8_t *row = nullptr;
+                float *srow = nullptr;
+                if (PEER) {
+                    if (nd.x >= 0) {
+                        row = a.peer_recv[nd.x] + (size_t)nd.y * a.H;
+                        if (a.peer_scales != nullptr) srow = a.peer_scales[nd.x] + (int64_t)nd.y * a.s_row;
+                    }
+                } else if (np >= 0) {
+                    row = a.recv + (size_t)np * a.H;
+                    if (a.scales != nullptr) srow = a.scales + (int64_t)np * a.s_row;
+                }
+                row_s[cur ^ 1][tid] = row;
+                srow_s[cur ^ 1][tid] = srow;
+            }
+            if (tid == 0) tok_s[cur ^ 1] = a.tok_scales != nullptr ? a.tok_scales + (int64_t)tn * G : nullptr;
+        }
+        cur ^= 1;
+    }
+}
+
 // Pre-quantised FP8 input: codes and scales are copied, not recomputed.
 template <bool LOOP, bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) {
@@ -280,7 +403,7 @@ cudaError_t launch_dispatch_impl(const DispatchArgs &a, cudaStream_t st) {
     const bool loop = a.num_sms > 0;
     void (*kernel)(DispatchArgs) =
         a.mode == kDispatchQuantFp8
-            ? (loop ? dispatch_fp8_kernel<true, PEER> : dispatch_fp8_kernel<false, PEER>)
+            ? (loop ? dispatch_fp8_loop_kernel<PEER> : dispatch_fp8_kernel<false, PEER>)
         : a.mode == kDispatchCopyFp8
             ? (loop ? dispatch_fp8_copy_kernel<true, PEER> : dispatch_fp8_copy_kernel<false, PEER>)
             : (loop ? dispatch_bf16_kernel<true, PEER> : dispatch_bf16_kernel<false, PEER>);
