@@ -60,8 +60,8 @@ REFERENCE_BUDGET_S = float(os.environ.get("EP_BENCH_REFERENCE_BUDGET_S", "150"))
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch each on the
     # metric workload (one ncu capture per kernel, keyed to the kernel source)
-    ("group_limited", "combine"): {"sha": "79eb048b8ac6c125", "bytes": 940067584 + 72227328},
-    ("group_limited", "dispatch"): {"sha": "aa2ecec9c00a91c0", "bytes": 117774848 + 425984768},
+    ("group_limited", "combine"): {"sha": "61964820f31d742f", "bytes": 940124416 + 72721408},
+    ("group_limited", "dispatch"): {"sha": "6e11ef9cfd0d0561", "bytes": 117787136 + 425800448},
 }
 
 
