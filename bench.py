@@ -61,7 +61,7 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch each on the
     # metric workload (one ncu capture per kernel, keyed to the kernel source)
     ("group_limited", "combine"): {"sha": "61964820f31d742f", "bytes": 940124416 + 72721408},
-    ("group_limited", "dispatch"): {"sha": "6e11ef9cfd0d0561", "bytes": 117787136 + 425800448},
+    ("group_limited", "dispatch"): {"sha": "70e5e8aacbf867c8", "bytes": 117771776 + 425458432},
 }
 
 

@@ -118,10 +118,12 @@ __device__ __forceinline__ void slot_rows(const DispatchArgs &a, int t, size_t r
     srow_s[j] = srow;
 }
 
-// The kernels take one (token, chunk) unit per block; when the caller caps
-// the grid (num_sms) the LOOP instantiation walks the units with a grid stride.
+// The FP8 kernels below take one (token, chunk) unit per block (the grid is
+// the unit count); a grid capped by the caller (num_sms) runs the pipelined
+// grid-stride kernels further down instead.  The BF16 kernel keeps a plain
+// grid stride (LOOP) for a capped grid.
 
-template <bool LOOP, bool PEER>
+template <bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
     __shared__ uint8_t *row_s[kMaxTopk];
     __shared__ float *srow_s[kMaxTopk];
@@ -133,8 +135,8 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
 #endif
     const int tid = threadIdx.x;
     const bool leader = (tid & 7) == 0;
-    // One unit per block unless the grid is capped (LOOP): then a grid stride.
-    for (int u = blockIdx.x; u < a.nunits; u += gridDim.x) {
+    {
+        const int u = blockIdx.x;
         const int t = u / a.nchunks;
         const int ch0 = (u - t * a.nchunks) * a.chunk;
         const int chn = min(a.chunk, a.H - ch0);
@@ -185,8 +187,6 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchArgs a) {
                 if (leader && srow_s[j] != nullptr) srow_s[j][(int64_t)g * a.s_grp] = scale;
             }
         }
-        if (!LOOP) break;
-        __syncthreads();  // row_s is rewritten by the next unit
     }
 }
 
@@ -313,8 +313,96 @@ __global__ void __launch_bounds__(512) dispatch_fp8_loop_kernel(DispatchArgs a) 
     }
 }
 
+// The same pipelining for pre-quantised FP8 input (codes and scales copied):
+// the next unit's codes, scales and row positions are loaded before this
+// unit's stores; same store pattern as dispatch_fp8_copy_kernel.  (BF16
+// copies keep the plain grid stride: pipelined, the kernel needs more than
+// 32 registers and loses a resident block per SM, which measured slower.)
+template <bool PEER>
+__global__ void __launch_bounds__(512) dispatch_fp8_copy_loop_kernel(DispatchArgs a) {
+    __shared__ uint8_t *row_s[2][kMaxTopk];
+    __shared__ float *srow_s[2][kMaxTopk];
+#if EP_DISPATCH_EARLY_TRIGGER
+    pdl_wait_then_trigger();
+#else
+    pdl_wait();
+#endif
+    const int tid = threadIdx.x;
+    const bool leader = (tid & 7) == 0;
+    const int G = a.H / 128;
+    // Codes and scale of unit u for this thread (zero past the chunk).
+    auto load_unit = [&](int u, uint4 &v, float &sc) {
+        v = make_uint4(0u, 0u, 0u, 0u);
+        sc = 0.0f;
+        const int t = u / a.nchunks;
+        const int ch = (u - t * a.nchunks) * a.chunk + tid * 16;
+        if (tid * 16 < min(a.chunk, a.H - (ch - tid * 16))) {
+            v = ld_nc_v4(a.x + (int64_t)t * a.H + ch);
+            if (leader) sc = __ldg(a.x_scales + (int64_t)t * G + ch / 128);
+        }
+    };
+    int u = blockIdx.x;
+    if (u >= a.nunits) return;
+    uint4 v;
+    float sc;
+    load_unit(u, v, sc);
+    slot_rows<PEER>(a, u / a.nchunks, (size_t)a.H, row_s[0], srow_s[0]);
+    int cur = 0;
+#pragma unroll 1
+    for (; u < a.nunits; u += gridDim.x) {
+        __syncthreads();  // buffer cur is published; nobody reads buffer cur ^ 1 any more
+        const int t = u / a.nchunks;
+        const int ch0 = (u - t * a.nchunks) * a.chunk;
+        const int ch = ch0 + tid * 16;
+        const bool act = tid * 16 < min(a.chunk, a.H - ch0);
+        const uint4 q = v;  // this unit's codes and scale
+        const float scale = sc;
+        // The next unit's loads, issued before this unit's stores.
+        const int un = u + gridDim.x;
+        const bool more = un < a.nunits;
+        const int tn = more ? un / a.nchunks : 0;
+        int np = -1;
+        int2 nd = make_int2(-1, -1);
+        if (more) {
+            load_unit(un, v, sc);
+            if (tid < a.k) {
+                if (PEER)
+                    nd = __ldg(a.dst + (int64_t)tn * a.k + tid);
+                else
+                    np = __ldg(a.pos + (int64_t)tn * a.k + tid);
+            }
+        }
+        if (act) {
+            const int g = ch / 128;
+            for (int j = 0; j < a.k; ++j) {
+                uint8_t *row = row_s[cur][j];
+                if (row == nullptr) continue;
+                st_row_v4(row + ch, q);
+                if (leader && srow_s[cur][j] != nullptr) srow_s[cur][j][(int64_t)g * a.s_grp] = scale;
+            }
+        }
+        // The next unit's row pointers, into the other buffer.
+        if (more && tid < a.k) {
+            uint8_t *row = nullptr;
+            float *srow = nullptr;
+            if (PEER) {
+                if (nd.x >= 0) {
+                    row = a.peer_recv[nd.x] + (size_t)nd.y * a.H;
+                    if (a.peer_scales != nullptr) srow = a.peer_scales[nd.x] + (int64_t)nd.y * a.s_row;
+                }
+            } else if (np >= 0) {
+                row = a.recv + (size_t)np * a.H;
+                if (a.scales != nullptr) srow = a.scales + (int64_t)np * a.s_row;
+            }
+            row_s[cur ^ 1][tid] = row;
+            srow_s[cur ^ 1][tid] = srow;
+        }
+        cur ^= 1;
+    }
+}
+
 // Pre-quantised FP8 input: codes and scales are copied, not recomputed.
-template <bool LOOP, bool PEER>
+template <bool PEER>
 __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) {
     __shared__ uint8_t *row_s[kMaxTopk];
     __shared__ float *srow_s[kMaxTopk];
@@ -326,8 +414,8 @@ __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) 
     const int tid = threadIdx.x;
     const bool leader = (tid & 7) == 0;
     const int G_row = a.H / 128;
-    // One unit per block unless the grid is capped (LOOP): then a grid stride.
-    for (int u = blockIdx.x; u < a.nunits; u += gridDim.x) {
+    {
+        const int u = blockIdx.x;
         const int t = u / a.nchunks;
         const int ch0 = (u - t * a.nchunks) * a.chunk;
         const int chn = min(a.chunk, a.H - ch0);
@@ -350,8 +438,6 @@ __global__ void __launch_bounds__(512) dispatch_fp8_copy_kernel(DispatchArgs a) 
                 if (leader && srow_s[j] != nullptr) srow_s[j][(int64_t)g * a.s_grp] = scale;
             }
         }
-        if (!LOOP) break;
-        __syncthreads();  // row_s is rewritten by the next unit
     }
 }
 
@@ -403,9 +489,9 @@ cudaError_t launch_dispatch_impl(const DispatchArgs &a, cudaStream_t st) {
     const bool loop = a.num_sms > 0;
     void (*kernel)(DispatchArgs) =
         a.mode == kDispatchQuantFp8
-            ? (loop ? dispatch_fp8_loop_kernel<PEER> : dispatch_fp8_kernel<false, PEER>)
+            ? (loop ? dispatch_fp8_loop_kernel<PEER> : dispatch_fp8_kernel<PEER>)
         : a.mode == kDispatchCopyFp8
-            ? (loop ? dispatch_fp8_copy_kernel<true, PEER> : dispatch_fp8_copy_kernel<false, PEER>)
+            ? (loop ? dispatch_fp8_copy_loop_kernel<PEER> : dispatch_fp8_copy_kernel<PEER>)
             : (loop ? dispatch_bf16_kernel<true, PEER> : dispatch_bf16_kernel<false, PEER>);
     int grid = a.nunits;
     if (loop) {
