@@ -106,6 +106,47 @@ def test_sm_budget_changes_nothing(num_sms):
         assert (u16(o0) == oracle.combine(y.cpu(), tw.numpy(), L.pos)).all()
 
 
+@pytest.mark.parametrize("num_sms", [1, 3])
+def test_sm_budget_pipelined_kernels_against_the_oracle(num_sms):
+    """The grid-stride kernels an SM budget runs (the next unit's inputs are
+    loaded while the current unit is stored, row pointers double-buffered)
+    against the oracle itself: FP8 quantising and pre-quantised dispatch, BF16
+    dispatch and combine, with two chunks per token (H = 8320 > 8192
+    channels), unused slots, a token with no slot and a padded layout, so
+    that every block walks many units of both chunk positions."""
+    w = W.WORKLOADS["prefill"].scaled(T=700, H=8192 + 128)
+    x, idx, tw = W.make_routing(w)
+    idx = idx.clone()
+    idx[::4, 2] = -1
+    idx[9, :] = -1
+    for C in (0, 96):
+        res = ep.ep_layout(idx.to(DEV), w.E, w.R, 1, C)
+        st, L = oracle.layout(idx.numpy(), w.E, w.R, 1, C)
+        assert st == 0
+        h = res.handle
+        rows = h.num_recv_rows
+        valid = L.src_idx >= 0
+        xd = x.to(DEV)
+        recv, sc, _ = ep.ep_dispatch_ex(h, xd, True, num_sms=num_sms)
+        xq, xs = oracle.quantize_rows(x)
+        rq, sq, _ = ep.ep_dispatch_ex(h, torch.from_numpy(xq).to(DEV).view(torch.float8_e4m3fn), True,
+                                      x_scales=torch.from_numpy(xs).to(DEV), num_sms=num_sms)
+        rb, _, _ = ep.ep_dispatch_ex(h, xd, False, num_sms=num_sms)
+        y = W.make_expert_out(rows, w.H, seed=7).to(DEV)
+        out = ep.ep_combine_ex(h, y, tw.to(DEV), num_sms=num_sms)
+        torch.cuda.synchronize()
+        q, s = oracle.dispatch_fp8(x, L.pos, L.n_rows)
+        assert (u8(recv)[valid] == q[valid]).all(), C
+        assert (sc.cpu().numpy()[valid].view(np.uint32) == s[valid].view(np.uint32)).all(), C
+        q2, s2 = oracle.dispatch_fp8_prequant(xq, xs, L.pos, L.n_rows)
+        assert (u8(rq)[valid] == q2[valid]).all(), C
+        assert (sq.cpu().numpy()[valid].view(np.uint32) == s2[valid].view(np.uint32)).all(), C
+        b = oracle.dispatch_bf16(x, L.pos, L.n_rows)
+        assert (u16(rb)[valid] == b[valid]).all(), C
+        assert (u16(out) == oracle.combine(y.cpu(), tw.numpy(), L.pos)).all(), C
+        h.free()
+
+
 def test_option_errors():
     w, x, tw, res, L = setup("prefill", 64)
     h = res.handle
