@@ -106,20 +106,22 @@ def test_sm_budget_changes_nothing(num_sms):
         assert (u16(o0) == oracle.combine(y.cpu(), tw.numpy(), L.pos)).all()
 
 
-@pytest.mark.parametrize("num_sms", [1, 3])
-def test_sm_budget_pipelined_kernels_against_the_oracle(num_sms):
+@pytest.mark.parametrize("num_sms,T,H,k", [(1, 700, 8192 + 128, 8), (3, 700, 8192 + 128, 8),
+                                            (2, 300, 1024, 32), (5, 333, 640, 1)])
+def test_sm_budget_pipelined_kernels_against_the_oracle(num_sms, T, H, k):
     """The grid-stride kernels an SM budget runs (the next unit's inputs are
     loaded while the current unit is stored, row pointers double-buffered)
     against the oracle itself: FP8 quantising and pre-quantised dispatch, BF16
-    dispatch and combine, with two chunks per token (H = 8320 > 8192
-    channels), unused slots, a token with no slot and a padded layout, so
-    that every block walks many units of both chunk positions."""
-    w = W.WORKLOADS["prefill"].scaled(T=700, H=8192 + 128)
+    dispatch and combine, with unused slots, a token with no slot and a
+    padded layout; two chunks per token (H = 8320 > 8192 channels), so that
+    every block walks many units of both chunk positions, and the extremes of
+    top-k (32 slots: the whole first warp loads positions; 1 slot)."""
+    w = W.WORKLOADS["prefill"].scaled(T=T, H=H, k=k)
     x, idx, tw = W.make_routing(w)
     idx = idx.clone()
-    idx[::4, 2] = -1
+    idx[::4, min(2, k - 1)] = -1
     idx[9, :] = -1
-    for C in (0, 96):
+    for C in (0, 96 if k > 1 else 8):
         res = ep.ep_layout(idx.to(DEV), w.E, w.R, 1, C)
         st, L = oracle.layout(idx.numpy(), w.E, w.R, 1, C)
         assert st == 0
